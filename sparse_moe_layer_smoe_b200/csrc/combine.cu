@@ -1,0 +1,79 @@
+// Combine: out[t] = y[T*k + t] + sum_j w[t, j] * y[perm_row[t*k + j]].
+// Source: every token's layer output is its shared-expert output plus the weighted outputs
+// of its 8 routed experts (Step 3.5 Flash summary, hyper.ai, section "方法"; weights from the
+// router, model card fields norm_expert_weight and moe_router_scaling_factor).
+//
+// One CTA per token; each thread owns 8 consecutive features (one 16-byte vector per row).
+// Accumulation is fp32 in slot order j = 0..k-1, the shared row is added last, and the sum is
+// rounded once to bf16. Rows outside [0, T*k) are skipped and set SMOE_ERR_DEVICE.
+#include "common.cuh"
+#include "internal.h"
+
+namespace smoe {
+
+namespace {
+
+constexpr int kMaxK = 32;
+
+__device__ __forceinline__ void fma8(float (&acc)[8], float w, const uint4 v) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = fmaf(w, __uint_as_float(u[i] << 16), acc[2 * i]);
+        acc[2 * i + 1] = fmaf(w, __uint_as_float(u[i] & 0xFFFF0000u), acc[2 * i + 1]);
+    }
+}
+
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y,
+                                                      const int32_t* __restrict__ perm_row,
+                                                      const float* __restrict__ topk_w, int T, int k, int H,
+                                                      uint16_t* __restrict__ out, int32_t* err) {
+    __shared__ int32_t rows[kMaxK];
+    __shared__ float ws[kMaxK];
+    const int t = blockIdx.x;
+    const int64_t nrouted = (int64_t)T * k;
+    if (threadIdx.x < k) {
+        int32_t r = perm_row[(size_t)t * k + threadIdx.x];
+        if (r < 0 || r >= nrouted) {
+            record_error(err, SMOE_ERR_DEVICE);
+            r = -1;
+        }
+        rows[threadIdx.x] = r;
+        ws[threadIdx.x] = topk_w[(size_t)t * k + threadIdx.x];
+    }
+    __syncthreads();
+    const int vec = H / 8;
+    const uint4* y4 = reinterpret_cast<const uint4*>(y);
+    for (int c = threadIdx.x; c < vec; c += blockDim.x) {
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        for (int j = 0; j < k; ++j) {
+            const int r = rows[j];
+            if (r >= 0) fma8(acc, ws[j], y4[(size_t)r * vec + c]);
+        }
+        fma8(acc, 1.0f, y4[(size_t)(nrouted + t) * vec + c]);
+        uint4 o;
+        uint32_t* ou = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            ou[i] = (uint32_t)float_to_bf16_bits(acc[2 * i]) | ((uint32_t)float_to_bf16_bits(acc[2 * i + 1]) << 16);
+        reinterpret_cast<uint4*>(out)[(size_t)t * vec + c] = o;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const smoe_config_t& c, const uint16_t* y, const int32_t* perm_row, const float* topk_w,
+                           int64_t T, uint16_t* out, int32_t* err, cudaStream_t s) {
+    const int threads = c.hidden / 8 >= 256 ? 256 : 128;
+    {
+        LaunchTimer lt(K_COMBINE, s);
+        combine_kernel<<<(unsigned)T, threads, 0, s>>>(y, perm_row, topk_w, (int)T, c.top_k, c.hidden, out, err);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) launches_add(1);
+    return e;
+}
+
+}  // namespace smoe

@@ -1,0 +1,81 @@
+// Internal interface between the C-ABI entry points (api.cu) and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/stepmoe.h"
+
+namespace smoe {
+
+constexpr size_t kAlign = 256;
+constexpr int kPermuteTokensPerBlock = 256;
+constexpr int kRouterKChunk = 32;
+
+inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
+
+// Router tiling for T tokens: tokens per CTA, experts per CTA, K splits.
+struct RouterPlan {
+    int tm, te, splits;
+};
+RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms);
+
+// Workspace: [error word | scratch union | forward intermediates]
+struct WsLayout {
+    size_t err = 0;
+    size_t scratch = 0;          // start of the scratch union
+    size_t route_partials = 0;   // [splits][T][E] fp32  (inside the union)
+    size_t perm_hist = 0;        // [nblk][E] int32      (inside the union)
+    size_t perm_base = 0;        // [nblk][E] int32      (inside the union)
+    size_t ffn_h = 0;            // [T*k + T][I] bf16    (inside the union)
+    size_t scratch_end = 0;
+    size_t topk_idx = 0, topk_w = 0, counts = 0, offsets = 0, perm_row = 0, row_token = 0, x_perm = 0, y = 0;
+    size_t total = 0;
+};
+WsLayout ws_layout(const smoe_config_t& c, int64_t T, int num_sms);
+
+int num_sms_current_device();
+
+// Per-thread count of kernels enqueued by the last entry point.
+void launches_reset();
+void launches_add(int n);
+
+// Per-kernel CUDA-event timing (smoe_timing_begin / smoe_timing_end). Each launcher wraps its
+// kernel launches in a LaunchTimer; when timing is off this is one branch.
+enum KernelId {
+    K_ROUTER_LOGITS = 0, K_ROUTER_TOPK, K_PERMUTE_HIST, K_PERMUTE_SCAN, K_PERMUTE_SCATTER, K_GATHER_ROWS,
+    K_EXPERT_GATEUP, K_EXPERT_DOWN, K_COMBINE, K_PACK_GATEUP, K_PACK_DOWN, K_NUM_KERNELS
+};
+const char* kernel_name(int id);
+
+struct LaunchTimer {
+    int slot = -1;
+    cudaStream_t stream = nullptr;
+    LaunchTimer(KernelId id, cudaStream_t s);
+    ~LaunchTimer();   // records the end event after the launch statement(s) in scope
+};
+
+cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, const float* wr, const float* bias,
+                         int32_t* topk_idx, float* topk_w, float* logits_opt, float* partials, int32_t* err,
+                         int num_sms, cudaStream_t s);
+
+cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int64_t T, const uint16_t* x,
+                           int32_t* counts, int32_t* offsets, int32_t* perm_row, int32_t* row_token,
+                           uint16_t* x_perm, int32_t* hist, int32_t* base, int32_t* err, cudaStream_t s);
+
+// Returns cudaErrorNotSupported when the driver entry point for tensor maps is unavailable.
+cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const uint16_t* x_perm,
+                              const int32_t* offsets, int64_t T, const void* packed, uint16_t* y, uint16_t* h,
+                              int32_t* err, int num_sms, cudaStream_t s);
+
+cudaError_t launch_combine(const smoe_config_t& c, const uint16_t* y, const int32_t* perm_row, const float* topk_w,
+                           int64_t T, uint16_t* out, int32_t* err, cudaStream_t s);
+
+cudaError_t launch_pack(const smoe_config_t& c, const uint16_t* wg, const uint16_t* wu, const uint16_t* wd,
+                        const uint16_t* sg, const uint16_t* su, const uint16_t* sd, void* packed, cudaStream_t s);
+
+size_t packed_gateup_bytes(const smoe_config_t& c);
+size_t packed_down_bytes(const smoe_config_t& c);
+
+}  // namespace smoe

@@ -1,0 +1,209 @@
+// Token -> expert dispatch: per-block expert histograms, a column scan, and a stable scatter
+// that orders rows by expert, then token, then slot (a unique order, so the result is
+// bit-exact and independent of scheduling), plus an optional gather of x into x_perm.
+//
+// Source: sparse top-k routing, Step 3.5 Flash summary (hyper.ai), section "方法" (method):
+// each token is sent to 8 of 288 routed experts; the grouping by expert is what the grouped
+// expert GEMMs consume.
+//
+// Kernels:
+//   permute_hist_kernel    block b counts entries of tokens [256 b, 256 b + 256) per expert
+//   permute_scan_kernel    one CTA: per-expert exclusive scan over blocks, counts, offsets
+//   permute_scatter_kernel rank of (t, e) among the block's tokens that chose e: per-warp
+//                          lane bitmasks in shared memory (a token picks an expert at most
+//                          once), warp prefix over the block, block base from the scan
+//   gather_rows_kernel     x_perm[r] = x[row_token[r]], one warp per row, 16-byte accesses
+// An expert id outside [0, E) or repeated within a token is skipped (perm_row = -1) and
+// recorded as SMOE_ERR_DEVICE.
+#include "common.cuh"
+#include "internal.h"
+
+namespace smoe {
+
+namespace {
+
+constexpr int TB = kPermuteTokensPerBlock;   // tokens per block = threads per block
+constexpr int WARPS = TB / 32;
+
+// Entry (t, j) is valid when its expert is in range and not already chosen at an earlier slot.
+__device__ __forceinline__ bool entry_valid(const int32_t* idx, int t, int j, int k, int E, int32_t* err) {
+    const int e = idx[(size_t)t * k + j];
+    if (e < 0 || e >= E) {
+        record_error(err, SMOE_ERR_DEVICE);
+        return false;
+    }
+    for (int q = 0; q < j; ++q) {
+        if (idx[(size_t)t * k + q] == e) {
+            record_error(err, SMOE_ERR_DEVICE);
+            return false;
+        }
+    }
+    return true;
+}
+
+__global__ void __launch_bounds__(TB) permute_hist_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
+                                                          int32_t* __restrict__ hist, int32_t* err) {
+    extern __shared__ int32_t sh[];
+    for (int e = threadIdx.x; e < E; e += TB) sh[e] = 0;
+    __syncthreads();
+    const int t = blockIdx.x * TB + threadIdx.x;
+    if (t < T) {
+        for (int j = 0; j < k; ++j)
+            if (entry_valid(idx, t, j, k, E, err)) atomicAdd(&sh[idx[(size_t)t * k + j]], 1);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += TB) hist[(size_t)blockIdx.x * E + e] = sh[e];
+}
+
+// One CTA of 1024 threads: base[b][e] = sum_{b' < b} hist[b'][e]; counts[e]; offsets = scan.
+__global__ void __launch_bounds__(1024) permute_scan_kernel(const int32_t* __restrict__ hist, int nblk, int E,
+                                                            int32_t* __restrict__ base, int32_t* __restrict__ counts,
+                                                            int32_t* __restrict__ offsets) {
+    __shared__ int32_t warp_tot[32];
+    const int e = threadIdx.x;
+    int32_t run = 0;
+    if (e < E) {
+        for (int b = 0; b < nblk; ++b) {
+            base[(size_t)b * E + e] = run;
+            run += hist[(size_t)b * E + e];
+        }
+        counts[e] = run;
+    }
+    // exclusive scan of run over e (E <= 1024)
+    const int lane = e & 31, w = e >> 5;
+    int32_t v = run;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int32_t n = __shfl_up_sync(0xFFFFFFFFu, v, off);
+        if (lane >= off) v += n;
+    }
+    if (lane == 31) warp_tot[w] = v;
+    __syncthreads();
+    if (w == 0) {
+        int32_t tv = warp_tot[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int32_t n = __shfl_up_sync(0xFFFFFFFFu, tv, off);
+            if (lane >= off) tv += n;
+        }
+        warp_tot[lane] = tv;   // inclusive totals of warps 0..lane
+    }
+    __syncthreads();
+    const int32_t incl = v + (w > 0 ? warp_tot[w - 1] : 0);
+    if (e < E) offsets[e] = incl - run;
+    if (e == E - 1) offsets[E] = incl;
+}
+
+__global__ void __launch_bounds__(TB) permute_scatter_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
+                                                             const int32_t* __restrict__ base,
+                                                             const int32_t* __restrict__ offsets,
+                                                             int32_t* __restrict__ perm_row,
+                                                             int32_t* __restrict__ row_token, int32_t* err) {
+    extern __shared__ uint32_t smem[];
+    uint32_t* wmask = smem;                                        // [WARPS][E]
+    int32_t* wbase = reinterpret_cast<int32_t*>(smem + WARPS * E);  // [WARPS][E]
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < WARPS * E; i += TB) wmask[i] = 0u;
+    __syncthreads();
+    const int t = blockIdx.x * TB + threadIdx.x;
+    if (t < T) {
+        for (int j = 0; j < k; ++j) {
+            // duplicates/out-of-range are recorded by the histogram pass; skip them silently here
+            const int e = idx[(size_t)t * k + j];
+            bool ok = (e >= 0 && e < E);
+            for (int q = 0; ok && q < j; ++q) ok = idx[(size_t)t * k + q] != e;
+            if (ok) atomicOr(&wmask[w * E + e], 1u << lane);
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += TB) {
+        int32_t run = offsets[e] + base[(size_t)blockIdx.x * E + e];
+        for (int q = 0; q < WARPS; ++q) {
+            wbase[q * E + e] = run;
+            run += __popc(wmask[q * E + e]);
+        }
+    }
+    __syncthreads();
+    if (t < T) {
+        const uint32_t below = (1u << lane) - 1u;
+        for (int j = 0; j < k; ++j) {
+            const int e = idx[(size_t)t * k + j];
+            bool ok = (e >= 0 && e < E);
+            for (int q = 0; ok && q < j; ++q) ok = idx[(size_t)t * k + q] != e;
+            int32_t row = -1;
+            if (ok) {
+                row = wbase[w * E + e] + __popc(wmask[w * E + e] & below);
+                row_token[row] = t;
+            }
+            perm_row[(size_t)t * k + j] = row;
+        }
+    }
+    (void)err;
+}
+
+// x_perm[r] = x[row_token[r]] for r < offsets[E]; one warp per row.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,
+                                                          const int32_t* __restrict__ row_token,
+                                                          const int32_t* __restrict__ offsets, int E, int T, int H,
+                                                          uint16_t* __restrict__ x_perm, int32_t* err) {
+    const int nrows = offsets[E];
+    const int lane = threadIdx.x & 31;
+    const int vec = H / 8;
+    for (int r = blockIdx.x * 8 + (threadIdx.x >> 5); r < nrows; r += gridDim.x * 8) {
+        const int t = row_token[r];
+        if (t < 0 || t >= T) {
+            if (lane == 0) record_error(err, SMOE_ERR_DEVICE);
+            continue;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+        uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * H);
+        for (int c = lane; c < vec; c += 32) dst[c] = src[c];
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int64_t T, const uint16_t* x,
+                           int32_t* counts, int32_t* offsets, int32_t* perm_row, int32_t* row_token,
+                           uint16_t* x_perm, int32_t* hist, int32_t* base, int32_t* err, cudaStream_t s) {
+    const int E = c.n_experts, k = c.top_k;
+    const int nblk = (int)((T + TB - 1) / TB);
+    {
+        LaunchTimer lt(K_PERMUTE_HIST, s);
+        permute_hist_kernel<<<nblk, TB, E * sizeof(int32_t), s>>>(topk_idx, (int)T, k, E, hist, err);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    {
+        LaunchTimer lt(K_PERMUTE_SCAN, s);
+        permute_scan_kernel<<<1, 1024, 0, s>>>(hist, nblk, E, base, counts, offsets);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const size_t sm = 2 * WARPS * E * sizeof(uint32_t);
+    if (sm > 48 * 1024) {
+        e = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+    }
+    {
+        LaunchTimer lt(K_PERMUTE_SCATTER, s);
+        permute_scatter_kernel<<<nblk, TB, sm, s>>>(topk_idx, (int)T, k, E, base, offsets, perm_row, row_token, err);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    int n = 3;
+    if (x != nullptr && x_perm != nullptr) {
+        const int64_t rows = T * k;
+        int64_t blocks = (rows + 7) / 8;
+        if (blocks > 148 * 8) blocks = 148 * 8;
+        {
+            LaunchTimer lt(K_GATHER_ROWS, s);
+            gather_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, row_token, offsets, E, (int)T, c.hidden, x_perm,
+                                                                err);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        ++n;
+    }
+    launches_add(n);
+    return cudaSuccess;
+}
+
+}  // namespace smoe

@@ -1,0 +1,305 @@
+// Router: fp32 logits L = x W_r^T (x bf16, upcast exactly), sigmoid scores s, biased scores
+// s + bias for selection, top-k, weights route_scale * s_j / sum s_j.
+//
+// Source: Step-3.5-Flash model card (llm-atlas), raw config fields need_fp32_gate,
+// moe_router_activation sigmoid, use_moe_router_bias, moe_top_k 8, norm_expert_weight,
+// moe_router_scaling_factor 3; the bias steers selection only (Step 3.5 Flash summary,
+// paperlayer.ai, §4.1.2: loss-free bias adjustment as the balancing device).
+//
+// Kernel 1 (router_logits_kernel): a register-tiled fp32 SGEMM on the CUDA cores. Each CTA
+// owns TM tokens x TE experts over one K range; K is split only when T is small, so the
+// 4.7 MB of W_r is spread over all SMs at decode sizes. Partial sums go to the workspace.
+// Kernel 2 (router_topk_kernel): one warp per token adds the K-split partials in a fixed
+// order (deterministic), applies sigmoid and bias, selects top-k by repeated warp argmax
+// with the tie rule (biased score, then larger logit, then smaller index) and normalises.
+#include <float.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace smoe {
+
+namespace {
+
+template <int TM, int TE, int RM, int RE>
+struct RouterTile {
+    static constexpr int TX = TE / RE;          // threads along experts
+    static constexpr int TY = TM / RM;          // threads along tokens
+    static constexpr int THREADS = TX * TY;
+    static constexpr int KC = kRouterKChunk;    // K elements per stage
+    static constexpr int XCHUNKS = TM * KC / 8; // 16-byte chunks of x per stage
+    static constexpr int WCHUNKS = TE * KC / 4; // 16-byte chunks of W_r per stage
+    static constexpr int XPT = (XCHUNKS + THREADS - 1) / THREADS;
+    static constexpr int WPT = (WCHUNKS + THREADS - 1) / THREADS;
+};
+
+template <int TM, int TE, int RM, int RE>
+__global__ void __launch_bounds__(RouterTile<TM, TE, RM, RE>::THREADS)
+router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr, float* __restrict__ part,
+                     int T, int E, int H, int k_len) {
+    using P = RouterTile<TM, TE, RM, RE>;
+    constexpr int KC = P::KC;
+    // +1 padding: the transposing stores below hit 32 distinct banks
+    __shared__ float xs[2][KC][TM + 1];
+    __shared__ float ws[2][KC][TE + 1];
+
+    const int tid = threadIdx.x;
+    const int tx = tid % P::TX, ty = tid / P::TX;
+    const int t0 = blockIdx.x * TM, e0 = blockIdx.y * TE;
+    const int kbeg = blockIdx.z * k_len;
+    const int nchunks = k_len / KC;
+
+    uint4 xr[P::XPT];
+    float4 wrg[P::WPT];
+
+    auto gload = [&](int kc) {
+        const int kb = kbeg + kc * KC;
+#pragma unroll
+        for (int i = 0; i < P::XPT; ++i) {
+            const int c = tid + i * P::THREADS;
+            xr[i] = make_uint4(0, 0, 0, 0);
+            if (c < P::XCHUNKS) {
+                const int m = c / (KC / 8), q = c % (KC / 8);
+                const int t = t0 + m;
+                if (t < T) xr[i] = *reinterpret_cast<const uint4*>(x + (size_t)t * H + kb + q * 8);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < P::WPT; ++i) {
+            const int c = tid + i * P::THREADS;
+            wrg[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (c < P::WCHUNKS) {
+                const int n = c / (KC / 4), q = c % (KC / 4);
+                const int e = e0 + n;
+                if (e < E) wrg[i] = *reinterpret_cast<const float4*>(wr + (size_t)e * H + kb + q * 4);
+            }
+        }
+    };
+    auto sstore = [&](int buf) {
+#pragma unroll
+        for (int i = 0; i < P::XPT; ++i) {
+            const int c = tid + i * P::THREADS;
+            if (c < P::XCHUNKS) {
+                const int m = c / (KC / 8), q = c % (KC / 8);
+                const uint32_t w4[4] = {xr[i].x, xr[i].y, xr[i].z, xr[i].w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    xs[buf][q * 8 + 2 * h][m] = __uint_as_float(w4[h] << 16);
+                    xs[buf][q * 8 + 2 * h + 1][m] = __uint_as_float(w4[h] & 0xFFFF0000u);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < P::WPT; ++i) {
+            const int c = tid + i * P::THREADS;
+            if (c < P::WCHUNKS) {
+                const int n = c / (KC / 4), q = c % (KC / 4);
+                ws[buf][q * 4 + 0][n] = wrg[i].x;
+                ws[buf][q * 4 + 1][n] = wrg[i].y;
+                ws[buf][q * 4 + 2][n] = wrg[i].z;
+                ws[buf][q * 4 + 3][n] = wrg[i].w;
+            }
+        }
+    };
+
+    float acc[RM][RE];
+#pragma unroll
+    for (int i = 0; i < RM; ++i)
+#pragma unroll
+        for (int j = 0; j < RE; ++j) acc[i][j] = 0.f;
+
+    gload(0);
+    sstore(0);
+    __syncthreads();
+    for (int kc = 0; kc < nchunks; ++kc) {
+        const int buf = kc & 1;
+        if (kc + 1 < nchunks) gload(kc + 1);
+#pragma unroll 8
+        for (int kk = 0; kk < KC; ++kk) {
+            float a[RM], b[RE];
+#pragma unroll
+            for (int i = 0; i < RM; ++i) a[i] = xs[buf][kk][ty * RM + i];
+#pragma unroll
+            for (int j = 0; j < RE; ++j) b[j] = ws[buf][kk][tx * RE + j];
+#pragma unroll
+            for (int i = 0; i < RM; ++i)
+#pragma unroll
+                for (int j = 0; j < RE; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        if (kc + 1 < nchunks) sstore(buf ^ 1);
+        __syncthreads();
+    }
+
+    float* dst = part + (size_t)blockIdx.z * T * E;
+#pragma unroll
+    for (int i = 0; i < RM; ++i) {
+        const int t = t0 + ty * RM + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < RE; ++j) {
+            const int e = e0 + tx * RE + j;
+            if (e < E) dst[(size_t)t * E + e] = acc[i][j];
+        }
+    }
+}
+
+// (b, l, e) is better than (b2, l2, e2): larger biased score, then larger logit, then
+// smaller expert index. NaN scores were mapped to -inf before, so the order is total.
+__device__ __forceinline__ bool better(float b, float l, int e, float b2, float l2, int e2) {
+    if (b != b2) return b > b2;
+    if (l != l2) return l > l2;
+    return e < e2;
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(256)
+router_topk_kernel(const float* __restrict__ part, int splits, const float* __restrict__ bias, int T, int E, int k,
+                   float scale, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                   float* __restrict__ logits_out) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+
+    float L[NPL], S[NPL], B[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        L[i] = -FLT_MAX;
+        S[i] = 0.f;
+        B[i] = -INFINITY;
+        if (e < E) {
+            float l = 0.f;
+            for (int s = 0; s < splits; ++s) l += part[((size_t)s * T + t) * E + e];
+            L[i] = l;
+            if (logits_out) logits_out[(size_t)t * E + e] = l;
+            const float sg = 1.0f / (1.0f + expf(-l));
+            S[i] = sg;
+            float bb = sg + bias[e];
+            B[i] = (bb != bb) ? -INFINITY : bb;
+            if (l != l) L[i] = -FLT_MAX;
+        }
+    }
+
+    uint32_t taken = 0;
+    float s_sel = 0.f;   // this lane's copy of the chosen score for slot j == lane
+    int e_sel = 0;
+    for (int j = 0; j < k; ++j) {
+        float bb = -INFINITY, ll = -FLT_MAX;
+        int ee = 0x7FFFFFFF;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !((taken >> i) & 1u) && better(B[i], L[i], e, bb, ll, ee)) {
+                bb = B[i];
+                ll = L[i];
+                ee = e;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float b2 = __shfl_xor_sync(0xFFFFFFFFu, bb, off);
+            const float l2 = __shfl_xor_sync(0xFFFFFFFFu, ll, off);
+            const int e2 = __shfl_xor_sync(0xFFFFFFFFu, ee, off);
+            if (better(b2, l2, e2, bb, ll, ee)) {
+                bb = b2;
+                ll = l2;
+                ee = e2;
+            }
+        }
+        // every lane now holds the winner ee (valid: k <= E, so an untaken expert exists)
+        float sw = 0.f;
+        if ((ee & 31) == lane) {
+            const int i = ee >> 5;
+#pragma unroll
+            for (int q = 0; q < NPL; ++q)
+                if (q == i) {
+                    taken |= 1u << q;
+                    sw = S[q];
+                }
+        }
+        sw = __shfl_sync(0xFFFFFFFFu, sw, ee & 31);
+        if (lane == j) {
+            s_sel = sw;
+            e_sel = ee;
+        }
+    }
+    // sum of the selected unbiased scores in slot order j = 0..k-1
+    float sum = 0.f;
+    for (int j = 0; j < k; ++j) sum += __shfl_sync(0xFFFFFFFFu, s_sel, j);
+    if (lane < k) {
+        topk_idx[(size_t)t * k + lane] = e_sel;
+        topk_w[(size_t)t * k + lane] = scale * (s_sel / sum);
+    }
+}
+
+template <int TM, int TE, int RM, int RE>
+cudaError_t launch_logits(const uint16_t* x, int64_t T, const float* wr, int E, int H, int splits, float* part,
+                          cudaStream_t s) {
+    using P = RouterTile<TM, TE, RM, RE>;
+    dim3 grid((unsigned)((T + TM - 1) / TM), (unsigned)((E + TE - 1) / TE), (unsigned)splits);
+    {
+        LaunchTimer lt(K_ROUTER_LOGITS, s);
+        router_logits_kernel<TM, TE, RM, RE><<<grid, P::THREADS, 0, s>>>(x, wr, part, (int)T, E, H, H / splits);
+    }
+    return cudaGetLastError();
+}
+
+template <int NPL>
+cudaError_t launch_topk(const float* part, int splits, const float* bias, int64_t T, int E, int k, float scale,
+                        int32_t* idx, float* w, float* logits, cudaStream_t s) {
+    const int warps = 8;
+    {
+        LaunchTimer lt(K_ROUTER_TOPK, s);
+        router_topk_kernel<NPL><<<(unsigned)((T + warps - 1) / warps), warps * 32, 0, s>>>(part, splits, bias, (int)T,
+                                                                                           E, k, scale, idx, w, logits);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms) {
+    RouterPlan p;
+    if (T >= 512) {
+        p.tm = 64;
+        p.te = (c.n_experts % 96 == 0) ? 96 : 64;
+    } else {
+        p.tm = 16;
+        p.te = 32;
+    }
+    const int64_t base = ((T + p.tm - 1) / p.tm) * ((c.n_experts + p.te - 1) / p.te);
+    const int chunks = c.hidden / kRouterKChunk;
+    int splits = 1;
+    while (splits * 2 <= 16 && chunks % (splits * 2) == 0 && base * splits * 2 <= 2 * (int64_t)num_sms) splits *= 2;
+    p.splits = splits;
+    return p;
+}
+
+cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, const float* wr, const float* bias,
+                         int32_t* topk_idx, float* topk_w, float* logits_opt, float* partials, int32_t* err,
+                         int num_sms, cudaStream_t s) {
+    (void)err;
+    const RouterPlan p = router_plan(c, T, num_sms);
+    const int E = c.n_experts, H = c.hidden;
+    cudaError_t e;
+    if (p.tm == 64 && p.te == 96)
+        e = launch_logits<64, 96, 4, 6>(x, T, wr, E, H, p.splits, partials, s);
+    else if (p.tm == 64)
+        e = launch_logits<64, 64, 4, 4>(x, T, wr, E, H, p.splits, partials, s);
+    else
+        e = launch_logits<16, 32, 2, 2>(x, T, wr, E, H, p.splits, partials, s);
+    if (e != cudaSuccess) return e;
+    const int npl = (E + 31) / 32;
+    if (npl <= 4)
+        e = launch_topk<4>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, s);
+    else if (npl <= 9)
+        e = launch_topk<9>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, s);
+    else if (npl <= 16)
+        e = launch_topk<16>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, s);
+    else
+        e = launch_topk<32>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, s);
+    if (e == cudaSuccess) launches_add(2);
+    return e;
+}
+
+}  // namespace smoe
