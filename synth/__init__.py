@@ -226,6 +226,9 @@ WORKLOADS = {
                        description="T=4096, Zipf(1.2) expert popularity via router bias, 16 dead experts"),
     "mtp": Workload("mtp", 512, 4096, 288, 8, 1280, 1280, spike_rows=5,
                     description="MTP-3 verify batch 128x4=512 tokens, 1% of rows x50"),
+    # profiling case: the decode kernel shape (~2 rows per expert) on 32 experts, ~1 GB of weights
+    "decode_e32": Workload("decode_e32", 8, 4096, 32, 8, 1280, 1280,
+                           description="decode-shaped small case for counter captures: T=8, 32 experts top-8"),
 }
 ZIPF_DEAD = 16
 ZIPF_FIXTURE = os.path.join(REPO, "tests", "golden", "zipf_bias.json")
