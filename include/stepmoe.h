@@ -190,6 +190,23 @@ SMOE_API smoe_status_t smoe_timing_begin(int32_t max_launches);
  * (at most cap entries) to out, their number to *n, and destroy the events. */
 SMOE_API smoe_status_t smoe_timing_end(smoe_kernel_time_t* out, int32_t cap, int32_t* n);
 
+/* Allocation-free router, for callers that cannot allocate device memory: a plugin that an
+ * inference runtime hands only its input and output buffers, or a serving path where
+ * cudaMalloc is forbidden after start-up because it can synchronise the device and stall.
+ * The pages have no counterpart to this entry point; it exists only for such callers.
+ * Same arguments and results as smoe_route, without the workspace. Its scratch (the router's
+ * K-split partial logits: splits x T x E x 4 bytes, 9.4 MB at T = 8192, E = 288) is a static
+ * device array of SMOE_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until the
+ * process exits; a T that needs more returns SMOE_ERR_WORKSPACE before any launch. The first
+ * call on each device looks up the array's device address (cudaGetSymbolAddress, with that
+ * device current); make that first call before any stream capture. Every call shares the one
+ * array and keeps nothing from earlier calls: calls that overlap on the GPU (several streams or
+ * host threads) race on it, so the caller must serialise them. Allocates and frees nothing. */
+#define SMOE_NOALLOC_SCRATCH_BYTES (16u << 20)
+SMOE_API smoe_status_t smoe_route_noalloc(const smoe_config_t* cfg, const smoe_bf16_t* x, int64_t T,
+                                          const float* w_router, const float* bias, int32_t* topk_idx,
+                                          float* topk_w, float* logits_opt, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

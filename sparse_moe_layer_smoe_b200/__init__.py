@@ -63,6 +63,7 @@ _SIGS = {
     "smoe_timing_begin": ([ctypes.c_int32], ctypes.c_int),
     "smoe_timing_end": ([ctypes.POINTER(SmoeKernelTime), ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)],
                         ctypes.c_int),
+    "smoe_route_noalloc": ([_cfgp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
 }
 
 _lib = None
@@ -147,6 +148,12 @@ def smoe_pack_weights(cfg, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, packed
 def smoe_route(cfg, x, T, w_router, bias, topk_idx, topk_w, logits=None, ws=None, ws_bytes=None, stream=None):
     _check("smoe_route", lib().smoe_route(ctypes.byref(cfg), _p(x), T, _p(w_router), _p(bias), _p(topk_idx),
                                           _p(topk_w), _p(logits), _p(ws), _ws_bytes(ws, ws_bytes), _s(stream)))
+
+
+def smoe_route_noalloc(cfg, x, T, w_router, bias, topk_idx, topk_w, logits=None, stream=None):
+    """smoe_route without a workspace (library-owned static scratch; see include/stepmoe.h)."""
+    _check("smoe_route_noalloc", lib().smoe_route_noalloc(ctypes.byref(cfg), _p(x), T, _p(w_router), _p(bias),
+                                                          _p(topk_idx), _p(topk_w), _p(logits), _s(stream)))
 
 
 def smoe_permute(cfg, topk_idx, T, x, counts, offsets, perm_row, row_token, x_perm, ws=None, ws_bytes=None,
