@@ -35,7 +35,8 @@ struct TimingState {
 const char* const kNames[K_NUM_KERNELS] = {"router_logits", "router_topk",   "permute_hist",
                                            "permute_scan",  "permute_scatter", "gather_rows",
                                            "expert_gateup", "expert_down",   "combine",
-                                           "pack_gateup",   "pack_down"};
+                                           "pack_gateup",   "pack_down",     "router_split",
+                                           "router_gemm"};
 }  // namespace
 
 const char* kernel_name(int id) { return (id >= 0 && id < K_NUM_KERNELS) ? kNames[id] : "unknown"; }
@@ -71,7 +72,7 @@ WsLayout ws_layout(const smoe_config_t& c, int64_t T, int num_sms) {
     const int64_t nblk = (T + kPermuteTokensPerBlock - 1) / kPermuteTokensPerBlock;
     L.err = 0;
     L.scratch = kAlign;
-    const size_t route_b = align_up((size_t)rp.splits * T * E * 4);
+    const size_t route_b = align_up(rp.scratch_bytes);
     const size_t perm_b = 2 * align_up((size_t)nblk * E * 4);
     const size_t h_b = align_up((size_t)(routed + T) * I * 2);
     L.route_partials = L.scratch;

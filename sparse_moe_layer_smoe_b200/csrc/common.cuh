@@ -191,18 +191,22 @@ __device__ __forceinline__ void tmem_ld2_x16_wait(uint32_t ta, uint32_t tb, uint
         : "memory");
 }
 
-// Shared-memory matrix descriptor for a K-major bf16 tile stored with the 128-byte swizzle
-// that TMA's SWIZZLE_128B mode writes: rows of 128 bytes, 8-row atoms 1024 bytes apart.
-//   bits  0-13 start address >> 4, 16-29 leading byte offset >> 4 (unused for this layout),
-//   bits 32-45 stride byte offset >> 4 (1024: next 8-row atom), bit 46 descriptor version 1,
-//   bits 49-51 base offset 0 (atoms are 1024-aligned), bits 61-63 layout 2 = 128B swizzle.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+// Shared-memory matrix descriptor for a K-major bf16 tile in the swizzled layout TMA writes
+// with SWIZZLE_{32,64,128}B: rows of SW bytes (SW/2 bf16 along K), 8-row atoms of 8*SW bytes.
+//   bits  0-13 start address >> 4, 16-29 leading byte offset >> 4 (unused for these layouts, 1),
+//   bits 32-45 stride byte offset >> 4 (8*SW: the next 8-row atom), bit 46 descriptor version 1,
+//   bits 49-51 base offset 0 (atoms are aligned), bits 61-63 layout: 2 = 128B, 4 = 64B, 6 = 32B.
+// A K-step of 16 bf16 inside the atom is selected by adding 32 bytes to the start address.
+template <int SW>
+__device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr) {
+    static_assert(SW == 32 || SW == 64 || SW == 128, "swizzle span");
+    constexpr uint64_t layout = SW == 128 ? 2 : (SW == 64 ? 4 : 6);
     uint64_t d = 0;
     d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
     d |= (uint64_t)(16u >> 4) << 16;
-    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)((8u * SW) >> 4) << 32;
     d |= (uint64_t)1 << 46;
-    d |= (uint64_t)2 << 61;
+    d |= layout << 61;
     return d;
 }
 

@@ -14,15 +14,19 @@
 //
 // Groups 0..E-1: routed experts, rows offsets[g] .. offsets[g+1] of the permuted activations.
 // Group E: the shared expert over all T rows (x for gate/up, the last T rows of h for down).
+// Token tile per group: the smallest power of two >= the group's row count, between 16 and a
+// launch-wide maximum NT_MAX (so an expert with 2 tokens runs N=16 MMAs while a hot expert with
+// 1000 tokens runs N=256 tiles). One TMA tensor map per tile height loads exactly that box.
 // Work unit = (group, 128-feature block mb, token tile nb), enumerated group-major, then mb,
 // then nb; CTA i takes units i, i + grid, ... (static persistent schedule, grid = #SMs).
 //
-// Roles (192 threads): warp 0 lane 0 issues TMA loads into an S-stage ring; warp 1 lane 0
-// issues tcgen05.mma (M=128, N=NT, K=16 per instruction, 4 per 64-wide stage; for gate/up a
-// second MMA into the neighbouring TMEM columns) and commits stage and accumulator barriers;
-// warps 2-5 drain the accumulator (tcgen05.ld, warp w reads TMEM lanes 32*(w%4)..+31),
-// apply SiLU(g)*u or pass through, round to bf16 and store. Accumulators are double-buffered
-// in TMEM whenever two fit in 512 columns, so the epilogue overlaps the next unit's MMAs.
+// Roles (192 threads): warp 0 lane 0 issues TMA loads into an S-stage ring of BK-wide K slices
+// (BK = 64: 128-byte swizzled rows; the ring fills the 227 KB of shared memory);
+// warp 1 lane 0 issues tcgen05.mma (M=128, N=tile, K=16 per instruction; for gate/up a second
+// MMA into the neighbouring TMEM columns) and commits stage and accumulator barriers; warps 2-5
+// drain the accumulator (tcgen05.ld, warp w reads TMEM lanes 32*(w%4)..+31), apply SiLU(g)*u or
+// pass through, round to bf16 and store. Accumulators are double-buffered in TMEM whenever two
+// fit in 512 columns, so the epilogue overlaps the next unit's MMAs.
 #include <algorithm>
 #include <mutex>
 
@@ -33,23 +37,22 @@ namespace smoe {
 
 namespace {
 
-constexpr int kBK = 64;             // K elements per stage: 128 bytes of bf16 = one swizzle row
+#ifndef SMOE_GEMM_BK
+#define SMOE_GEMM_BK 64          // K elements per pipeline stage (16, 32 or 64): 64 measured fastest
+#endif
+#ifndef SMOE_MAX_TOKEN_TILE
+#define SMOE_MAX_TOKEN_TILE 256  // cap on the token tile (a tuning constant)
+#endif
+
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
-constexpr int kSmemBudget = 200 * 1024;
+constexpr int kNumTiles = 5;     // token tiles 16, 32, 64, 128, 256
+constexpr int kMaxStages = 24;
 
-template <int NT, bool DUAL>
-struct GemmCfg {
-    static constexpr int A_ROWS = DUAL ? 256 : 128;     // gate 128 + up 128, or 128
-    static constexpr int A_BYTES = A_ROWS * 128;
-    static constexpr int B_BYTES = NT * 128;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = (kSmemBudget / STAGE_BYTES) > 12 ? 12 : (kSmemBudget / STAGE_BYTES);
-    static constexpr int ACC_COLS = DUAL ? 2 * NT : NT;
-    static constexpr int NACC = (2 * ACC_COLS <= kTmemCols) ? 2 : 1;
-    static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "MMA N for M=128 is 16..256 in steps of 16");
-    static_assert(ACC_COLS <= kTmemCols, "accumulator must fit TMEM");
-    static_assert(STAGES >= 2, "need at least two stages");
+struct GemmMaps {
+    CUtensorMap w;                  // weights [rows][K]: box {BK, 256 (gate/up) or 128 (down)}
+    CUtensorMap act[kNumTiles];     // routed activations [T*k][K]: box {BK, 16 << i}
+    CUtensorMap sh[kNumTiles];      // shared-group activations: box {BK, 16 << i}
 };
 
 struct GemmParams {
@@ -61,51 +64,88 @@ struct GemmParams {
     int n_out;                // output features per group (= leading dimension of out)
     int shared_in_row;        // first activation row of the shared group in its tensor map
     int shared_out_row;       // first output row of the shared group (= T*k)
-    uint16_t* out;            // [*, n_out] bf16
+    int nt_max;               // largest token tile of this launch (16..256, power of two)
+    int stages;               // pipeline depth
+    int k_wrap;               // B's K coordinate wraps every k_wrap blocks (0 = no wrap)
+    int out_ld;               // leading dimension of the output rows
+    int out_valid;            // output features stored: f < out_valid
+    uint16_t* out;            // [*, out_ld] bf16 (gate/up, down)
+    float* out_f32;           // [*, out_ld] fp32 (router)
     int32_t* err;
 };
 
-template <int NT, bool DUAL>
-size_t gemm_smem_bytes(int E) {
-    using C = GemmCfg<NT, DUAL>;
-    size_t b = 1024;                                   // alignment slack
-    b += (size_t)C::STAGES * C::STAGE_BYTES;
-    b += sizeof(uint64_t) * (2 * C::STAGES + 5);       // full, empty, tfull[2], tempty[2], drain
-    b += 16;                                           // tmem slot, abort flag
-    b += sizeof(int32_t) * (2 * (size_t)E + 3);        // prefix[E+2], offs[E+1]
+// What a launch computes: the down projection, the fused gate/up + SiLU*mul, or router logits.
+enum GemmMode { MODE_DOWN = 0, MODE_GATEUP = 1, MODE_ROUTER = 2 };
+
+template <int MODE, int BK>
+struct GemmCfg {
+    static constexpr bool DUAL = MODE == MODE_GATEUP;
+    static constexpr int SW = BK * 2;                     // bytes per swizzled row
+    static constexpr int A_ROWS = DUAL ? 256 : 128;       // gate 128 + up 128, or 128
+    static constexpr int A_BYTES = A_ROWS * SW;
+    static constexpr int UP_OFFSET = 128 * SW;            // up rows inside the A tile
+    static_assert(BK == 16 || BK == 32 || BK == 64, "stage K width");
+};
+
+__host__ __device__ inline int stage_bytes(bool dual, int bk, int nt_max) {
+    return (dual ? 256 : 128) * bk * 2 + nt_max * bk * 2;
+}
+
+__host__ __device__ inline size_t gemm_smem_bytes(int stages, int stage_b, int E) {
+    size_t b = 1024;                                       // alignment slack
+    b += (size_t)stages * stage_b;
+    b += sizeof(uint64_t) * (2 * (size_t)stages + 5);      // full, empty, tfull[2], tempty[2], drain
+    b += 16;                                               // tmem slot, abort flag
+    b += sizeof(int32_t) * (2 * (size_t)E + 3);            // prefix[E+2], offs[E+1]
     return b;
 }
 
 struct Unit {
-    int g, mb, nb;
+    int g, mb, nb, nt;
 };
 
 __device__ __forceinline__ int group_rows(int g, int E, int T, const int32_t* offs) {
     return g < E ? offs[g + 1] - offs[g] : T;
 }
 
-__device__ __forceinline__ Unit decode_unit(int u, const int32_t* prefix, const int32_t* offs, int E, int T, int NT) {
+// Token tile of a group: smallest power of two >= rows, clamped to [16, nt_max].
+__device__ __forceinline__ int group_tile(int rows, int nt_max) {
+    int nt = 16;
+    while (nt < rows && nt < nt_max) nt <<= 1;
+    return nt;
+}
+
+__device__ __forceinline__ int tile_index(int nt) { return 31 - __clz(nt) - 4; }   // 16 -> 0 ... 256 -> 4
+
+__device__ __forceinline__ Unit decode_unit(int u, const int32_t* prefix, const int32_t* offs, int E, int T,
+                                            int nt_max) {
     int lo = 0, hi = E;   // find g with prefix[g] <= u < prefix[g+1]
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (prefix[mid] <= u) lo = mid; else hi = mid - 1;
     }
     const int g = lo;
-    const int nblk = (group_rows(g, E, T, offs) + NT - 1) / NT;
+    const int rows = group_rows(g, E, T, offs);
+    const int nt = group_tile(rows, nt_max);
+    const int nblk = (rows + nt - 1) / nt;
     const int local = u - prefix[g];
-    return Unit{g, local / nblk, local % nblk};
+    return Unit{g, local / nblk, local % nblk, nt};
 }
 
-template <int NT, bool DUAL>
+template <int MODE, int BK>
 __global__ void __launch_bounds__(kThreads, 1)
-expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_act,
-                   const __grid_constant__ CUtensorMap tm_sh, const GemmParams p) {
-    using C = GemmCfg<NT, DUAL>;
+expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
+    using C = GemmCfg<MODE, BK>;
+    constexpr bool DUAL = C::DUAL;
     extern __shared__ uint8_t smem_raw[];
+    const int S = p.stages;
+    const int STAGE_B = stage_bytes(DUAL, BK, p.nt_max);
+    const int ACC_COLS = DUAL ? 2 * p.nt_max : p.nt_max;
+    const int NACC = (2 * ACC_COLS <= kTmemCols) ? 2 : 1;
     uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(tiles + (size_t)C::STAGES * C::STAGE_BYTES);
-    uint64_t* empty = full + C::STAGES;
-    uint64_t* tfull = empty + C::STAGES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(tiles + (size_t)S * STAGE_B);
+    uint64_t* empty = full + S;
+    uint64_t* tfull = empty + S;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -116,10 +156,10 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
     const int MB = p.n_out / 128;
-    const int KB = p.K / kBK;
+    const int KB = p.K / BK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(smem_u32(&full[s]), 1);
             mbar_init(smem_u32(&empty[s]), 1);
         }
@@ -136,15 +176,18 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         tmem_relinquish();
     }
     if (warp == 1 && lane == 0) {
-        tma_prefetch_desc(&tm_w);
-        tma_prefetch_desc(&tm_act);
-        tma_prefetch_desc(&tm_sh);
+        tma_prefetch_desc(&maps.w);
+        for (int i = 0; i < kNumTiles; ++i)
+            if ((16 << i) <= p.nt_max) {
+                tma_prefetch_desc(&maps.act[i]);
+                tma_prefetch_desc(&maps.sh[i]);
+            }
     }
     if (warp == 2) {
         // group table: offsets (validated), then units per group and their exclusive prefix
         bool bad = false;
         for (int i = lane; i <= E; i += 32) {
-            int v = p.offsets[i];
+            int v = (p.offsets != nullptr) ? p.offsets[i] : 0;
             if (v < 0 || v > p.routed_rows) { bad = true; v = 0; }
             offs[i] = v;
         }
@@ -160,8 +203,13 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         const int ngroups = E + 1;
         const int chunk = (ngroups + 31) / 32;
         const int g0 = min(lane * chunk, ngroups), g1 = min(g0 + chunk, ngroups);
+        auto units_of = [&](int g) {
+            const int rows = group_rows(g, E, p.T, offs);
+            const int nt = group_tile(rows, p.nt_max);
+            return ((rows + nt - 1) / nt) * MB;
+        };
         int local = 0;
-        for (int g = g0; g < g1; ++g) local += ((group_rows(g, E, p.T, offs) + NT - 1) / NT) * MB;
+        for (int g = g0; g < g1; ++g) local += units_of(g);
         int incl = local;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -171,7 +219,7 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         int run = incl - local;
         for (int g = g0; g < g1; ++g) {
             prefix[g] = run;
-            run += ((group_rows(g, E, p.T, offs) + NT - 1) / NT) * MB;
+            run += units_of(g);
         }
         if (lane == 31) prefix[E + 1] = incl;
     }
@@ -189,53 +237,60 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         uint32_t phase = 0, armed = 0, armed_par = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
-            const Unit w = decode_unit(u, prefix, offs, E, p.T, NT);
+            const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
             const int a_row = DUAL ? (w.g * MB + w.mb) * 256 : w.g * p.n_out + w.mb * 128;
-            const int b_row = (w.g < E ? offs[w.g] : p.shared_in_row) + w.nb * NT;
-            const CUtensorMap* bm = (w.g < E) ? &tm_act : &tm_sh;
+            const int b_row = (w.g < E ? offs[w.g] : p.shared_in_row) + w.nb * w.nt;
+            const int ti = tile_index(w.nt);
+            const CUtensorMap* bm = (w.g < E) ? &maps.act[ti] : &maps.sh[ti];
+            const uint32_t tx = (uint32_t)(C::A_BYTES + w.nt * BK * 2);
             for (int kb = 0; kb < KB; ++kb) {
                 if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag, true)) { ok = false; break; }
                 const uint32_t fb = smem_u32(&full[stage]);
-                mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-                uint8_t* a_s = tiles + (size_t)stage * C::STAGE_BYTES;
-                tma_load_2d(smem_u32(a_s), &tm_w, kb * kBK, a_row, fb, pol_w);
-                tma_load_2d(smem_u32(a_s + C::A_BYTES), bm, kb * kBK, b_row, fb, pol_a);
+                mbar_arrive_expect_tx(fb, tx);
+                uint8_t* a_s = tiles + (size_t)stage * STAGE_B;
+                tma_load_2d(smem_u32(a_s), &maps.w, kb * BK, a_row, fb, pol_w);
+                const int b_k = p.k_wrap ? (kb % p.k_wrap) : kb;
+                tma_load_2d(smem_u32(a_s + C::A_BYTES), bm, b_k * BK, b_row, fb, pol_a);
                 armed |= 1u << stage;
                 armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-                if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+                if (++stage == S) { stage = 0; phase ^= 1u; }
             }
         }
         // every load issued must land before the CTA may exit
-        for (int s = 0; s < C::STAGES; ++s)
+        for (int s = 0; s < S; ++s)
             if ((armed >> s) & 1u) mbar_wait(smem_u32(&full[s]), (armed_par >> s) & 1u, p.err, abort_flag, false);
     } else if (warp == 1 && lane == 0) {
         // ---------------------------------------------------------------- MMA issuer
-        constexpr uint32_t idesc = idesc_bf16_f32(128, NT);
+        const uint32_t idesc0 = idesc_bf16_f32(128, 0);
         int stage = 0, acc = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
+            const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
+            const uint32_t idesc = idesc0 | ((uint32_t)(w.nt >> 3) << 17);
             if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, p.err, abort_flag, true)) break;
             tc_fence_after();
-            const uint32_t d = tmem_base + (uint32_t)(acc * C::ACC_COLS);
+            const uint32_t d = tmem_base + (uint32_t)(acc * ACC_COLS);
             for (int kb = 0; kb < KB; ++kb) {
                 if (!mbar_wait(smem_u32(&full[stage]), phase, p.err, abort_flag, true)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t a_s = smem_u32(tiles + (size_t)stage * C::STAGE_BYTES);
+                const uint32_t a_s = smem_u32(tiles + (size_t)stage * STAGE_B);
                 const uint32_t b_s = a_s + C::A_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk) {
+                for (int kk = 0; kk < BK / 16; ++kk) {
                     const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
-                    const uint64_t bdesc = smem_desc_sw128(b_s + kk * 32);
-                    umma_f16_ss(d, smem_desc_sw128(a_s + kk * 32), bdesc, idesc, accum);
-                    if (DUAL) umma_f16_ss(d + NT, smem_desc_sw128(a_s + 16384 + kk * 32), bdesc, idesc, accum);
+                    const uint64_t bdesc = smem_desc_kmajor<C::SW>(b_s + kk * 32);
+                    umma_f16_ss(d, smem_desc_kmajor<C::SW>(a_s + kk * 32), bdesc, idesc, accum);
+                    if (DUAL)
+                        umma_f16_ss(d + p.nt_max, smem_desc_kmajor<C::SW>(a_s + C::UP_OFFSET + kk * 32), bdesc, idesc,
+                                    accum);
                 }
                 umma_commit(smem_u32(&empty[stage]));
-                if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+                if (++stage == S) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
             umma_commit(smem_u32(&tfull[acc]));
-            if (C::NACC == 2) {
+            if (NACC == 2) {
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
             } else {
@@ -252,33 +307,40 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
-            const Unit w = decode_unit(u, prefix, offs, E, p.T, NT);
+            const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
             const int rows = group_rows(w.g, E, p.T, offs);
-            const int out_base = (w.g < E ? offs[w.g] : p.shared_out_row) + w.nb * NT;
-            const int nvalid = min(NT, rows - w.nb * NT);
+            const int out_base = (w.g < E ? offs[w.g] : p.shared_out_row) + w.nb * w.nt;
+            const int nvalid = min(w.nt, rows - w.nb * w.nt);
             if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.err, abort_flag, true)) break;
             tc_fence_after();
-            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
-            uint16_t* dst = p.out + (size_t)out_base * p.n_out + w.mb * 128 + row;
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+            const int f = w.mb * 128 + row;
+            const bool keep = f < p.out_valid;
+            const size_t dst0 = (size_t)out_base * p.out_ld + f;
             for (int c0 = 0; c0 < nvalid; c0 += 16) {
                 uint32_t g16[16], u16[16];
                 if (DUAL)
-                    tmem_ld2_x16_wait(t_row + c0, t_row + NT + c0, g16, u16);
+                    tmem_ld2_x16_wait(t_row + c0, t_row + p.nt_max + c0, g16, u16);
                 else
                     tmem_ld_x16_wait(t_row + c0, g16);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    if (c0 + j < nvalid) {
+                    if (c0 + j < nvalid && keep) {
                         const float gv = __uint_as_float(g16[j]);
-                        float v = gv;
-                        if (DUAL) v = (gv / (1.0f + expf(-gv))) * __uint_as_float(u16[j]);
-                        dst[(size_t)(c0 + j) * p.n_out] = float_to_bf16_bits(v);
+                        const size_t o = dst0 + (size_t)(c0 + j) * p.out_ld;
+                        if (MODE == MODE_ROUTER) {
+                            p.out_f32[o] = gv;
+                        } else {
+                            float v = gv;
+                            if (DUAL) v = (gv / (1.0f + expf(-gv))) * __uint_as_float(u16[j]);
+                            p.out[o] = float_to_bf16_bits(v);
+                        }
                     }
                 }
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&tempty[acc]));
-            if (C::NACC == 2) {
+            if (NACC == 2) {
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
             } else {
@@ -315,52 +377,76 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2D bf16 tensor [rows][cols] row-major; box = 64 columns (128 bytes) x box_rows, 128B swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// 2D bf16 tensor [rows][cols] row-major; box = BK columns (2*BK bytes, swizzled) x box_rows.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows, int bk) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)bk, box_rows};
     cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle sw = bk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                           : (bk == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NT, bool DUAL>
-cudaError_t run_gemm(const CUtensorMap& w, const CUtensorMap& act, const CUtensorMap& sh, const GemmParams& p,
-                     int grid, cudaStream_t s) {
-    const size_t smem = gemm_smem_bytes<NT, DUAL>(p.E);
-    cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<NT, DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+// Activation maps for every token tile up to nt_max (larger entries repeat a valid map, unused).
+bool make_act_maps(CUtensorMap* maps, const void* base, uint64_t rows, uint64_t cols, int nt_max, int bk) {
+    for (int i = 0; i < kNumTiles; ++i) {
+        const int nt = 16 << i;
+        if (nt <= nt_max) {
+            if (!make_map(&maps[i], base, rows, cols, nt, bk)) return false;
+        } else {
+            maps[i] = maps[i - 1];
+        }
+    }
+    return true;
+}
+
+int max_dynamic_smem() {
+    static int v = 0;
+    if (v == 0) {
+        int dev = 0, n = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess && n > 0)
+            v = n;
+        else
+            v = 227 * 1024;
+    }
+    return v;
+}
+
+template <int MODE>
+cudaError_t run_gemm(const GemmMaps& maps, GemmParams p, int grid, cudaStream_t s) {
+    constexpr int BK = SMOE_GEMM_BK;
+    constexpr bool DUAL = MODE == MODE_GATEUP;
+    const int sb = stage_bytes(DUAL, BK, p.nt_max);
+    const size_t fixed = gemm_smem_bytes(0, sb, p.E) + 2 * sizeof(uint64_t) * kMaxStages;
+    int stages = (int)((max_dynamic_smem() - fixed) / sb);
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages < 2) return cudaErrorInvalidConfiguration;
+    p.stages = stages;
+    const size_t smem = gemm_smem_bytes(stages, sb, p.E);
+    cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     {
-        LaunchTimer lt(DUAL ? K_EXPERT_GATEUP : K_EXPERT_DOWN, s);
-        expert_gemm_kernel<NT, DUAL><<<grid, kThreads, smem, s>>>(w, act, sh, p);
+        LaunchTimer lt(MODE == MODE_GATEUP ? K_EXPERT_GATEUP : (MODE == MODE_DOWN ? K_EXPERT_DOWN : K_ROUTER_GEMM), s);
+        expert_gemm_kernel<MODE, BK><<<grid, kThreads, smem, s>>>(maps, p);
     }
     return cudaGetLastError();
 }
 
-template <bool DUAL>
-cudaError_t dispatch_nt(int nt, const CUtensorMap& w, const CUtensorMap& act, const CUtensorMap& sh,
-                        const GemmParams& p, int grid, cudaStream_t s) {
-    switch (nt) {
-        case 16: return run_gemm<16, DUAL>(w, act, sh, p, grid, s);
-        case 32: return run_gemm<32, DUAL>(w, act, sh, p, grid, s);
-        case 64: return run_gemm<64, DUAL>(w, act, sh, p, grid, s);
-        case 128: return run_gemm<128, DUAL>(w, act, sh, p, grid, s);
-        default: return run_gemm<256, DUAL>(w, act, sh, p, grid, s);
-    }
-}
-
 }  // namespace
 
-// Token tile: the smallest power of two >= 1.25 x the mean rows per routed expert, 16..256.
+// Largest token tile of a launch: the smallest power of two >= 1.25 x the mean rows per routed
+// expert, 16..256. Groups with fewer rows use smaller tiles inside the kernel.
 int choose_token_tile(const smoe_config_t& c, int64_t T) {
     const double mean = (double)T * c.top_k / c.n_experts;
     int nt = 16;
-    while (nt < 256 && nt < 1.25 * mean) nt *= 2;
+    while (nt < SMOE_MAX_TOKEN_TILE && nt < 1.25 * mean) nt *= 2;
     return nt;
 }
 
@@ -372,26 +458,44 @@ size_t packed_down_bytes(const smoe_config_t& c) { return (size_t)(c.n_experts +
 cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const uint16_t* x_perm,
                               const int32_t* offsets, int64_t T, const void* packed, uint16_t* y, uint16_t* h,
                               int32_t* err, int num_sms, cudaStream_t s) {
+    constexpr int BK = SMOE_GEMM_BK;
     const int E = c.n_experts, H = c.hidden, I = c.inter, k = c.top_k;
     const int64_t routed = T * k;
     const int nt = choose_token_tile(c, T);
     const uint8_t* wgu = static_cast<const uint8_t*>(packed);
     const uint8_t* wdn = wgu + packed_gateup_bytes(c);
 
-    CUtensorMap m_wgu, m_xp, m_x, m_wd, m_h;
-    if (!make_map(&m_wgu, wgu, (uint64_t)(E + 1) * 2 * I, H, 256) ||
-        !make_map(&m_xp, x_perm, (uint64_t)routed, H, nt) || !make_map(&m_x, x, (uint64_t)T, H, nt) ||
-        !make_map(&m_wd, wdn, (uint64_t)(E + 1) * H, I, 128) ||
-        !make_map(&m_h, h, (uint64_t)(routed + T), I, nt))
+    GemmMaps m1, m2;
+    if (!make_map(&m1.w, wgu, (uint64_t)(E + 1) * 2 * I, H, 256, BK) ||
+        !make_act_maps(m1.act, x_perm, (uint64_t)routed, H, nt, BK) ||
+        !make_act_maps(m1.sh, x, (uint64_t)T, H, nt, BK) ||
+        !make_map(&m2.w, wdn, (uint64_t)(E + 1) * H, I, 128, BK) ||
+        !make_act_maps(m2.act, h, (uint64_t)(routed + T), I, nt, BK))
         return cudaErrorNotSupported;
+    for (int i = 0; i < kNumTiles; ++i) m2.sh[i] = m2.act[i];
 
-    GemmParams p1{offsets, E, (int)T, (int)routed, H, I, 0, (int)routed, h, err};
-    cudaError_t e = dispatch_nt<true>(nt, m_wgu, m_xp, m_x, p1, num_sms, s);
+    GemmParams p1{offsets, E, (int)T, (int)routed, H, I, 0, (int)routed, nt, 0, 0, I, I, h, nullptr, err};
+    cudaError_t e = run_gemm<MODE_GATEUP>(m1, p1, num_sms, s);
     if (e != cudaSuccess) return e;
-    GemmParams p2{offsets, E, (int)T, (int)routed, I, H, (int)routed, (int)routed, y, err};
-    e = dispatch_nt<false>(nt, m_wd, m_h, m_h, p2, num_sms, s);
+    GemmParams p2{offsets, E, (int)T, (int)routed, I, H, (int)routed, (int)routed, nt, 0, 0, H, H, y, nullptr, err};
+    e = run_gemm<MODE_DOWN>(m2, p2, num_sms, s);
     if (e == cudaSuccess) launches_add(2);
     return e;
+}
+
+// Router logits on the tensor cores: logits[T][E] = x [T][H] . (W_hi + W_mid + W_lo)^T, where
+// w_split [e_pad][3H] holds the three bf16 pieces of each fp32 router row side by side (rows
+// >= E are zero). One group of T rows; the K loop runs over 3H while x's K coordinate wraps.
+cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* w_split, int e_pad, int E,
+                               float* logits, int nt, int num_sms, cudaStream_t s) {
+    constexpr int BK = SMOE_GEMM_BK;
+    GemmMaps m;
+    if (!make_map(&m.w, w_split, (uint64_t)e_pad, (uint64_t)3 * H, 128, BK) ||
+        !make_act_maps(m.sh, x, (uint64_t)T, H, nt, BK))
+        return cudaErrorNotSupported;
+    for (int i = 0; i < kNumTiles; ++i) m.act[i] = m.sh[i];
+    GemmParams p{nullptr, 0, (int)T, 0, 3 * H, e_pad, 0, 0, nt, 0, H / BK, E, E, nullptr, logits, nullptr};
+    return run_gemm<MODE_ROUTER>(m, p, num_sms, s);
 }
 
 }  // namespace smoe

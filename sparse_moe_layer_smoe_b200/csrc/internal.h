@@ -15,11 +15,15 @@ constexpr int kRouterKChunk = 32;
 
 inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
 
-// Router tiling for T tokens: tokens per CTA, experts per CTA, K splits.
+// Router plan for T tokens. CUDA cores: tokens per CTA, experts per CTA, K splits. Tensor cores
+// (tc, large T): W_r split into three bf16 pieces in the workspace, token tile nt.
 struct RouterPlan {
     int tm, te, splits;
+    bool tc;
+    int nt, e_pad;
+    size_t scratch_bytes;   // partial logits (+ the split weights when tc)
 };
-RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms);
+RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms, bool allow_tc = true);
 
 // Workspace: [error word | scratch union | forward intermediates]
 struct WsLayout {
@@ -45,7 +49,8 @@ void launches_add(int n);
 // kernel launches in a LaunchTimer; when timing is off this is one branch.
 enum KernelId {
     K_ROUTER_LOGITS = 0, K_ROUTER_TOPK, K_PERMUTE_HIST, K_PERMUTE_SCAN, K_PERMUTE_SCATTER, K_GATHER_ROWS,
-    K_EXPERT_GATEUP, K_EXPERT_DOWN, K_COMBINE, K_PACK_GATEUP, K_PACK_DOWN, K_NUM_KERNELS
+    K_EXPERT_GATEUP, K_EXPERT_DOWN, K_COMBINE, K_PACK_GATEUP, K_PACK_DOWN, K_ROUTER_SPLIT, K_ROUTER_GEMM,
+    K_NUM_KERNELS
 };
 const char* kernel_name(int id);
 
@@ -58,7 +63,10 @@ struct LaunchTimer {
 
 cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, const float* wr, const float* bias,
                          int32_t* topk_idx, float* topk_w, float* logits_opt, float* partials, int32_t* err,
-                         int num_sms, cudaStream_t s);
+                         int num_sms, cudaStream_t s, bool allow_tc = true);
+
+cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* w_split, int e_pad, int E,
+                               float* logits, int nt, int num_sms, cudaStream_t s);
 
 cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int64_t T, const uint16_t* x,
                            int32_t* counts, int32_t* offsets, int32_t* perm_row, int32_t* row_token,

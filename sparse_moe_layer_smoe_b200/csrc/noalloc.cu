@@ -61,14 +61,15 @@ extern "C" smoe_status_t smoe_route_noalloc(const smoe_config_t* c, const smoe_b
         if (p == nullptr || !aligned16(p)) return SMOE_ERR_INVALID_ARG;
     if (logits_opt != nullptr && !aligned16(logits_opt)) return SMOE_ERR_INVALID_ARG;
     const int sms = num_sms_current_device();
-    const RouterPlan rp = router_plan(*c, T, sms);
-    const size_t need = (size_t)rp.splits * (size_t)T * (size_t)c->n_experts * sizeof(float);
+    const RouterPlan rp = router_plan(*c, T, sms, /*allow_tc=*/false);
+    const size_t need = rp.scratch_bytes;
     if (need > (size_t)SMOE_NOALLOC_SCRATCH_BYTES) return SMOE_ERR_WORKSPACE;
     void* scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return SMOE_ERR_CUDA;
     // Every element of the partial-logit area the kernels read is written first in the same
     // call, so nothing needs clearing.
     const cudaError_t e = launch_route(*c, x, T, w_router, bias, topk_idx, topk_w, logits_opt,
-                                       static_cast<float*>(scratch), nullptr, sms, static_cast<cudaStream_t>(stream));
+                                       static_cast<float*>(scratch), nullptr, sms, static_cast<cudaStream_t>(stream),
+                                       /*allow_tc=*/false);
     return e == cudaSuccess ? SMOE_OK : SMOE_ERR_CUDA;
 }

@@ -6,9 +6,13 @@
 // moe_router_scaling_factor 3; the bias steers selection only (Step 3.5 Flash summary,
 // paperlayer.ai, §4.1.2: loss-free bias adjustment as the balancing device).
 //
-// Kernel 1 (router_logits_kernel): a register-tiled fp32 SGEMM on the CUDA cores. Each CTA
-// owns TM tokens x TE experts over one K range; K is split only when T is small, so the
+// Logits, small T (router_logits_kernel): a register-tiled fp32 SGEMM on the CUDA cores. Each
+// CTA owns TM tokens x TE experts over one K range; K is split only when T is small, so the
 // 4.7 MB of W_r is spread over all SMs at decode sizes. Partial sums go to the workspace.
+// Logits, large T (router_split_kernel + the grouped tensor-core GEMM in router mode): W_r is
+// split exactly into three bf16 pieces, so x W_r^T = x W_hi^T + x W_mid^T + x W_lo^T with
+// every product exact, accumulated in fp32 in TMEM (19 GFLOP of fp32 at T = 8192 become
+// 58 GFLOP of bf16 on the tensor cores).
 // Kernel 2 (router_topk_kernel): one warp per token adds the K-split partials in a fixed
 // order (deterministic), applies sigmoid and bias, selects top-k by repeated warp argmax
 // with the tie rule (biased score, then larger logit, then smaller index) and normalises.
@@ -232,6 +236,31 @@ router_topk_kernel(const float* __restrict__ part, int splits, const float* __re
     }
 }
 
+// W_split[e][p*H + h] = piece p (0 = hi, 1 = mid, 2 = lo) of W_r[e][h]: hi = bf16(w),
+// mid = bf16(w - hi), lo = bf16(w - hi - mid), each difference exact in fp32, so
+// hi + mid + lo reproduces w to about 2^-24 relative and every product with a bf16 x is exact
+// in fp32. Rows e >= E (padding up to a multiple of 128) are zero.
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ wr, int E, int e_pad, int H,
+                                                           uint16_t* __restrict__ w_split) {
+    const int64_t n = (int64_t)e_pad * H;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int e = (int)(i / H), h = (int)(i % H);
+        uint16_t p0 = 0, p1 = 0, p2 = 0;
+        if (e < E) {
+            const float w = wr[(size_t)e * H + h];
+            p0 = float_to_bf16_bits(w);
+            const float r1 = w - bf16_bits_to_float(p0);
+            p1 = float_to_bf16_bits(r1);
+            const float r2 = r1 - bf16_bits_to_float(p1);
+            p2 = float_to_bf16_bits(r2);
+        }
+        uint16_t* row = w_split + (size_t)e * 3 * H;
+        row[h] = p0;
+        row[H + h] = p1;
+        row[2 * H + h] = p2;
+    }
+}
+
 template <int TM, int TE, int RM, int RE>
 cudaError_t launch_logits(const uint16_t* x, int64_t T, const float* wr, int E, int H, int splits, float* part,
                           cudaStream_t s) {
@@ -258,36 +287,64 @@ cudaError_t launch_topk(const float* part, int splits, const float* bias, int64_
 
 }  // namespace
 
-RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms) {
-    RouterPlan p;
+// Tokens at which the router moves to the tensor cores (3-way bf16 split of W_r).
+constexpr int64_t kRouterTensorCoreMinT = 2048;
+
+RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms, bool allow_tc) {
+    RouterPlan p{};
+    const int E = c.n_experts;
+    if (allow_tc && T >= kRouterTensorCoreMinT) {
+        p.tc = true;
+        p.e_pad = (E + 127) / 128 * 128;
+        const int mb = p.e_pad / 128;
+        p.nt = 256;
+        while (p.nt > 64 && ((T + p.nt - 1) / p.nt) * mb < num_sms) p.nt /= 2;
+        p.splits = 1;
+        const size_t logit_b = ((size_t)T * E * 4 + 255) / 256 * 256;
+        p.scratch_bytes = logit_b + (size_t)p.e_pad * 3 * c.hidden * 2;
+        return p;
+    }
     if (T >= 512) {
         p.tm = 64;
-        p.te = (c.n_experts % 96 == 0) ? 96 : 64;
+        p.te = (E % 96 == 0) ? 96 : 64;
     } else {
         p.tm = 16;
         p.te = 32;
     }
-    const int64_t base = ((T + p.tm - 1) / p.tm) * ((c.n_experts + p.te - 1) / p.te);
+    const int64_t base = ((T + p.tm - 1) / p.tm) * ((E + p.te - 1) / p.te);
     const int chunks = c.hidden / kRouterKChunk;
     int splits = 1;
     while (splits * 2 <= 16 && chunks % (splits * 2) == 0 && base * splits * 2 <= 2 * (int64_t)num_sms) splits *= 2;
     p.splits = splits;
+    p.scratch_bytes = (size_t)splits * T * E * 4;
     return p;
 }
 
 cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, const float* wr, const float* bias,
                          int32_t* topk_idx, float* topk_w, float* logits_opt, float* partials, int32_t* err,
-                         int num_sms, cudaStream_t s) {
+                         int num_sms, cudaStream_t s, bool allow_tc) {
     (void)err;
-    const RouterPlan p = router_plan(c, T, num_sms);
+    const RouterPlan p = router_plan(c, T, num_sms, allow_tc);
     const int E = c.n_experts, H = c.hidden;
     cudaError_t e;
-    if (p.tm == 64 && p.te == 96)
+    int n = 2;
+    if (p.tc) {
+        const size_t logit_b = ((size_t)T * E * 4 + 255) / 256 * 256;
+        uint16_t* w_split = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(partials) + logit_b);
+        {
+            LaunchTimer lt(K_ROUTER_SPLIT, s);
+            router_split_kernel<<<148 * 4, 256, 0, s>>>(wr, E, p.e_pad, H, w_split);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch_router_gemm(x, T, H, w_split, p.e_pad, E, partials, p.nt, num_sms, s);
+        n = 3;
+    } else if (p.tm == 64 && p.te == 96) {
         e = launch_logits<64, 96, 4, 6>(x, T, wr, E, H, p.splits, partials, s);
-    else if (p.tm == 64)
+    } else if (p.tm == 64) {
         e = launch_logits<64, 64, 4, 4>(x, T, wr, E, H, p.splits, partials, s);
-    else
+    } else {
         e = launch_logits<16, 32, 2, 2>(x, T, wr, E, H, p.splits, partials, s);
+    }
     if (e != cudaSuccess) return e;
     const int npl = (E + 31) / 32;
     if (npl <= 4)
@@ -298,7 +355,7 @@ cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, c
         e = launch_topk<16>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, s);
     else
         e = launch_topk<32>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, s);
-    if (e == cudaSuccess) launches_add(2);
+    if (e == cudaSuccess) launches_add(n);
     return e;
 }
 
