@@ -122,7 +122,8 @@ SMOE_API smoe_status_t smoe_route(const smoe_config_t* cfg, const smoe_bf16_t* x
 /* Token -> expert dispatch: per-expert histogram, exclusive scan, stable scatter.
  *   topk_idx  [T][k] int32 (from smoe_route, or any selection of k distinct experts)
  *   counts    [E] int32 out: rows per expert
- *   offsets   [E+1] int32 out: exclusive scan of counts, offsets[E] = T*k
+ *   offsets   [E+1] int32 out: exclusive scan of counts (offsets[E] = T*k when every entry
+ *             is valid; skipped entries get perm_row = -1 and no row)
  *   perm_row  [T*k] int32 out: entry t*k+j -> its row; rows are expert-major, then token
  *             ascending, then slot ascending (a unique order, so results are bit-exact)
  *   row_token [T*k] int32 out: row -> token
@@ -134,14 +135,17 @@ SMOE_API smoe_status_t smoe_permute(const smoe_config_t* cfg, const int32_t* top
 
 /* Expert FFNs: grouped gate/up GEMM fused with SiLU-mul, then grouped down GEMM, on the
  * tensor cores (tcgen05, bf16 in, fp32 accumulate). Groups 0..E-1 are the routed experts
- * over their rows of x_perm; group E is the shared expert over all T rows of x.
- *   x         [T][H] bf16;  x_perm [T*k][H] bf16 (rows grouped by offsets)
- *   row_token [T*k] int32 (reserved for a gathering path; may be NULL)
+ * over their rows; group E is the shared expert over all T rows of x.
+ *   x         [T][H] bf16
+ *   x_perm    [T*k][H] bf16 rows grouped by offsets, or NULL: then the routed rows are read
+ *             straight from x through row_token (TMA row gathers; no permuted copy of x)
+ *   row_token [T*k] int32, as written by smoe_permute (needed when x_perm is NULL)
  *   offsets   [E+1] int32 (device), as written by smoe_permute
  *   packed    packed weights (smoe_pack_weights)
  *   y         [T*k + T][H] bf16 out: rows 0..T*k-1 routed (permuted order), rows T*k.. shared
  * The SwiGLU hidden h = SiLU(g) * u is computed in fp32 from fp32 accumulators and rounded
- * once to bf16 (kept in the workspace); y is rounded once to bf16. */
+ * once to bf16 (kept in the workspace); y is rounded once to bf16.
+ * Returns SMOE_ERR_INVALID_ARG when both x_perm and row_token are NULL. */
 SMOE_API smoe_status_t smoe_expert_ffn(const smoe_config_t* cfg, const smoe_bf16_t* x, const smoe_bf16_t* x_perm,
                               const int32_t* row_token, const int32_t* offsets, int64_t T, const void* packed,
                               smoe_bf16_t* y, void* ws, size_t ws_bytes, void* stream);
@@ -156,7 +160,9 @@ SMOE_API smoe_status_t smoe_combine(const smoe_config_t* cfg, const smoe_bf16_t*
                            void* stream);
 
 /* The whole layer: route -> permute -> expert_ffn -> combine on one stream, every
- * intermediate in the workspace (at least smoe_workspace_bytes(cfg, T) bytes).
+ * intermediate in the workspace (at least smoe_workspace_bytes(cfg, T) bytes). When the mean
+ * rows per expert are small (token tiles <= 32 rows) the expert GEMM gathers routed rows from
+ * x itself; otherwise permute writes the permuted copy x_perm into the workspace.
  *   x [T][H] bf16, w_router [E][H] fp32, bias [E] fp32, packed weights, out [T][H] bf16. */
 SMOE_API smoe_status_t smoe_forward(const smoe_config_t* cfg, const smoe_bf16_t* x, int64_t T, const float* w_router,
                            const float* bias, const void* packed, smoe_bf16_t* out, void* ws, size_t ws_bytes,

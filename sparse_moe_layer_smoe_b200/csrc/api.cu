@@ -87,7 +87,8 @@ WsLayout ws_layout(const smoe_config_t& c, int64_t T, int num_sms) {
     L.offsets = o;   o += align_up((size_t)(E + 1) * 4);
     L.perm_row = o;  o += align_up((size_t)routed * 4);
     L.row_token = o; o += align_up((size_t)routed * 4);
-    L.x_perm = o;    o += align_up((size_t)routed * H * 2);
+    L.x_perm = o;    // only when smoe_forward materialises the permuted rows (large token tiles)
+    if (choose_token_tile(c, T) > kGatherMaxTile) o += align_up((size_t)routed * H * 2);
     L.y = o;         o += align_up((size_t)(routed + T) * H * 2);
     L.total = o;
     return L;
@@ -255,16 +256,16 @@ smoe_status_t smoe_expert_ffn(const smoe_config_t* c, const smoe_bf16_t* x, cons
     launches_reset();
     if (T == 0) return SMOE_OK;
     SMOE_REQUIRE_PTR(x);
-    if (x_perm == nullptr) return SMOE_ERR_UNSUPPORTED;   // the row-gathering path is not built
-    SMOE_REQUIRE_PTR(x_perm);
+    SMOE_OPTIONAL_PTR(x_perm);
     SMOE_OPTIONAL_PTR(row_token);
+    if (x_perm == nullptr && row_token == nullptr) return SMOE_ERR_INVALID_ARG;   // one of the two is needed
     SMOE_REQUIRE_PTR(offsets);
     SMOE_REQUIRE_PTR(packed);
     SMOE_REQUIRE_PTR(y);
     SMOE_TRY(check_ws(c, T, ws, ws_bytes, false));
     const int sms = num_sms_current_device();
     const WsLayout L = ws_layout(*c, T, sms);
-    return cuda_status(launch_expert_ffn(*c, x, x_perm, offsets, T, packed, y, at<uint16_t>(ws, L.ffn_h),
+    return cuda_status(launch_expert_ffn(*c, x, x_perm, row_token, offsets, T, packed, y, at<uint16_t>(ws, L.ffn_h),
                                          at<int32_t>(ws, L.err), sms, static_cast<cudaStream_t>(stream)));
 }
 
@@ -306,15 +307,19 @@ smoe_status_t smoe_forward(const smoe_config_t* c, const smoe_bf16_t* x, int64_t
     float* w = at<float>(ws, L.topk_w);
     int32_t* offsets = at<int32_t>(ws, L.offsets);
     int32_t* perm_row = at<int32_t>(ws, L.perm_row);
-    uint16_t* x_perm = at<uint16_t>(ws, L.x_perm);
+    int32_t* row_token = at<int32_t>(ws, L.row_token);
     uint16_t* y = at<uint16_t>(ws, L.y);
     cudaError_t e = launch_route(*c, x, T, w_router, bias, idx, w, nullptr, at<float>(ws, L.route_partials), err,
                                  sms, s);
+    // small token tiles: routed rows are gathered from x inside the expert GEMM (no permuted
+    // copy); large tiles: one gather kernel writes x_perm and the GEMM loads whole tiles
+    const bool gather = choose_token_tile(*c, T) <= kGatherMaxTile;
+    uint16_t* x_perm = gather ? nullptr : at<uint16_t>(ws, L.x_perm);
     if (e == cudaSuccess)
-        e = launch_permute(*c, idx, T, x, at<int32_t>(ws, L.counts), offsets, perm_row, at<int32_t>(ws, L.row_token),
+        e = launch_permute(*c, idx, T, gather ? nullptr : x, at<int32_t>(ws, L.counts), offsets, perm_row, row_token,
                            x_perm, at<int32_t>(ws, L.perm_hist), at<int32_t>(ws, L.perm_base), err, s);
     if (e == cudaSuccess)
-        e = launch_expert_ffn(*c, x, x_perm, offsets, T, packed, y, at<uint16_t>(ws, L.ffn_h), err, sms, s);
+        e = launch_expert_ffn(*c, x, x_perm, row_token, offsets, T, packed, y, at<uint16_t>(ws, L.ffn_h), err, sms, s);
     if (e == cudaSuccess) e = launch_combine(*c, y, perm_row, w, T, out, err, s);
     return cuda_status(e);
 }

@@ -69,6 +69,7 @@ struct GemmParams {
     int k_wrap;               // B's K coordinate wraps every k_wrap blocks (0 = no wrap)
     int out_ld;               // leading dimension of the output rows
     int out_valid;            // output features stored: f < out_valid
+    const int32_t* row_token; // gather mode (routed groups read x rows by token), else nullptr
     uint16_t* out;            // [*, out_ld] bf16 (gate/up, down)
     float* out_f32;           // [*, out_ld] fp32 (router)
     int32_t* err;
@@ -229,8 +230,12 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     const uint32_t tmem_base = *tmem_slot;
     const int total = prefix[E + 1];
 
-    if (warp == 0 && lane == 0) {
-        // ---------------------------------------------------------------- TMA producer
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer (warp 0)
+        // Lane 0 waits for a free stage, arms its barrier and loads the weight tile. Activation
+        // rows come either as one tile (contiguous rows) or, for routed groups in gather mode,
+        // as token rows picked straight out of x by tile::gather4 loads that the 32 lanes share
+        // (4 rows each; rows past the group's end repeat its last row and are never stored).
         const uint64_t pol_w = l2_policy_evict_first();
         const uint64_t pol_a = l2_policy_evict_last();
         int stage = 0;
@@ -241,24 +246,55 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             const int a_row = DUAL ? (w.g * MB + w.mb) * 256 : w.g * p.n_out + w.mb * 128;
             const int b_row = (w.g < E ? offs[w.g] : p.shared_in_row) + w.nb * w.nt;
             const int ti = tile_index(w.nt);
-            const CUtensorMap* bm = (w.g < E) ? &maps.act[ti] : &maps.sh[ti];
+            const bool gather = p.row_token != nullptr && w.g < E;
+            const CUtensorMap* bm = (w.g < E) ? &maps.act[gather ? 0 : ti] : &maps.sh[ti];
             const uint32_t tx = (uint32_t)(C::A_BYTES + w.nt * BK * 2);
+            // gather mode: this lane's chunks of 4 rows (chunk c = lane + 32 j) and their tokens
+            int tok[8];
+            const int nchunks = w.nt / 4;
+            if (gather) {
+                const int last = offs[w.g + 1] - 1;
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int c = lane + 32 * j;
+                        const int r = min(b_row + 4 * c + i, last);
+                        tok[4 * j + i] = (c < nchunks) ? p.row_token[r] : 0;
+                    }
+            }
             for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag, true)) { ok = false; break; }
+                if (lane == 0) ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag, true);
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) break;
                 const uint32_t fb = smem_u32(&full[stage]);
-                mbar_arrive_expect_tx(fb, tx);
                 uint8_t* a_s = tiles + (size_t)stage * STAGE_B;
-                tma_load_2d(smem_u32(a_s), &maps.w, kb * BK, a_row, fb, pol_w);
                 const int b_k = p.k_wrap ? (kb % p.k_wrap) : kb;
-                tma_load_2d(smem_u32(a_s + C::A_BYTES), bm, b_k * BK, b_row, fb, pol_a);
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(fb, tx);
+                    tma_load_2d(smem_u32(a_s), &maps.w, kb * BK, a_row, fb, pol_w);
+                    if (!gather) tma_load_2d(smem_u32(a_s + C::A_BYTES), bm, b_k * BK, b_row, fb, pol_a);
+                }
+                __syncwarp();
+                if (gather) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int c = lane + 32 * j;
+                        if (c < nchunks)
+                            tma_gather4_2d(smem_u32(a_s + C::A_BYTES + c * 4 * BK * 2), bm, b_k * BK, tok[4 * j],
+                                           tok[4 * j + 1], tok[4 * j + 2], tok[4 * j + 3], fb, pol_a);
+                    }
+                }
                 armed |= 1u << stage;
                 armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                 if (++stage == S) { stage = 0; phase ^= 1u; }
             }
         }
         // every load issued must land before the CTA may exit
-        for (int s = 0; s < S; ++s)
-            if ((armed >> s) & 1u) mbar_wait(smem_u32(&full[s]), (armed_par >> s) & 1u, p.err, abort_flag, false);
+        if (lane == 0)
+            for (int s = 0; s < S; ++s)
+                if ((armed >> s) & 1u) mbar_wait(smem_u32(&full[s]), (armed_par >> s) & 1u, p.err, abort_flag, false);
+        __syncwarp();
     } else if (warp == 1 && lane == 0) {
         // ---------------------------------------------------------------- MMA issuer
         const uint32_t idesc0 = idesc_bf16_f32(128, 0);
@@ -456,8 +492,8 @@ size_t packed_gateup_bytes(const smoe_config_t& c) {
 size_t packed_down_bytes(const smoe_config_t& c) { return (size_t)(c.n_experts + 1) * c.hidden * c.inter * 2; }
 
 cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const uint16_t* x_perm,
-                              const int32_t* offsets, int64_t T, const void* packed, uint16_t* y, uint16_t* h,
-                              int32_t* err, int num_sms, cudaStream_t s) {
+                              const int32_t* row_token, const int32_t* offsets, int64_t T, const void* packed,
+                              uint16_t* y, uint16_t* h, int32_t* err, int num_sms, cudaStream_t s) {
     constexpr int BK = SMOE_GEMM_BK;
     const int E = c.n_experts, H = c.hidden, I = c.inter, k = c.top_k;
     const int64_t routed = T * k;
@@ -466,18 +502,24 @@ cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const u
     const uint8_t* wdn = wgu + packed_gateup_bytes(c);
 
     GemmMaps m1, m2;
-    if (!make_map(&m1.w, wgu, (uint64_t)(E + 1) * 2 * I, H, 256, BK) ||
-        !make_act_maps(m1.act, x_perm, (uint64_t)routed, H, nt, BK) ||
+    const bool gather = x_perm == nullptr;
+    bool ok_act = gather ? make_map(&m1.act[0], x, (uint64_t)T, H, 1, BK)
+                         : make_act_maps(m1.act, x_perm, (uint64_t)routed, H, nt, BK);
+    if (gather)
+        for (int i = 1; i < kNumTiles; ++i) m1.act[i] = m1.act[0];
+    if (!ok_act || !make_map(&m1.w, wgu, (uint64_t)(E + 1) * 2 * I, H, 256, BK) ||
         !make_act_maps(m1.sh, x, (uint64_t)T, H, nt, BK) ||
         !make_map(&m2.w, wdn, (uint64_t)(E + 1) * H, I, 128, BK) ||
         !make_act_maps(m2.act, h, (uint64_t)(routed + T), I, nt, BK))
         return cudaErrorNotSupported;
     for (int i = 0; i < kNumTiles; ++i) m2.sh[i] = m2.act[i];
 
-    GemmParams p1{offsets, E, (int)T, (int)routed, H, I, 0, (int)routed, nt, 0, 0, I, I, h, nullptr, err};
+    GemmParams p1{offsets, E, (int)T, (int)routed, H, I, 0, (int)routed, nt, 0, 0, I, I, gather ? row_token : nullptr,
+                  h, nullptr, err};
     cudaError_t e = run_gemm<MODE_GATEUP>(m1, p1, num_sms, s);
     if (e != cudaSuccess) return e;
-    GemmParams p2{offsets, E, (int)T, (int)routed, I, H, (int)routed, (int)routed, nt, 0, 0, H, H, y, nullptr, err};
+    GemmParams p2{offsets, E, (int)T, (int)routed, I, H, (int)routed, (int)routed, nt, 0, 0, H, H, nullptr, y, nullptr,
+                  err};
     e = run_gemm<MODE_DOWN>(m2, p2, num_sms, s);
     if (e == cudaSuccess) launches_add(2);
     return e;
@@ -494,7 +536,7 @@ cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16
         !make_act_maps(m.sh, x, (uint64_t)T, H, nt, BK))
         return cudaErrorNotSupported;
     for (int i = 0; i < kNumTiles; ++i) m.act[i] = m.sh[i];
-    GemmParams p{nullptr, 0, (int)T, 0, 3 * H, e_pad, 0, 0, nt, 0, H / BK, E, E, nullptr, logits, nullptr};
+    GemmParams p{nullptr, 0, (int)T, 0, 3 * H, e_pad, 0, 0, nt, 0, H / BK, E, E, nullptr, nullptr, logits, nullptr};
     return run_gemm<MODE_ROUTER>(m, p, num_sms, s);
 }
 

@@ -72,10 +72,18 @@ cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int6
                            int32_t* counts, int32_t* offsets, int32_t* perm_row, int32_t* row_token,
                            uint16_t* x_perm, int32_t* hist, int32_t* base, int32_t* err, cudaStream_t s);
 
+// Largest token tile of an expert-GEMM launch for T tokens (16..256).
+int choose_token_tile(const smoe_config_t& c, int64_t T);
+
+// smoe_forward reads routed rows straight from x (TMA row gathers) when the largest token tile
+// is at most this; above it, per-row gathers cost more than one gather kernel plus tile loads.
+constexpr int kGatherMaxTile = 32;
+
+// x_perm == nullptr selects gather mode: routed rows are read from x through row_token.
 // Returns cudaErrorNotSupported when the driver entry point for tensor maps is unavailable.
 cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const uint16_t* x_perm,
-                              const int32_t* offsets, int64_t T, const void* packed, uint16_t* y, uint16_t* h,
-                              int32_t* err, int num_sms, cudaStream_t s);
+                              const int32_t* row_token, const int32_t* offsets, int64_t T, const void* packed,
+                              uint16_t* y, uint16_t* h, int32_t* err, int num_sms, cudaStream_t s);
 
 cudaError_t launch_combine(const smoe_config_t& c, const uint16_t* y, const int32_t* perm_row, const float* topk_w,
                            int64_t T, uint16_t* out, int32_t* err, cudaStream_t s);

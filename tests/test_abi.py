@@ -55,8 +55,11 @@ def test_sizes():
     s1, s8 = smoe.smoe_scratch_bytes(c, 1), smoe.smoe_scratch_bytes(c, 8192)
     w8 = smoe.smoe_workspace_bytes(c, 8192)
     assert 0 < s1 < s8 < w8
-    # forward workspace holds at least x_perm and y
+    # forward workspace at T=8192 (large token tiles) holds x_perm and y; at T=64 (rows gathered
+    # from x inside the GEMM) no x_perm
     assert w8 >= 8192 * 8 * 4096 * 2 + (8192 * 9) * 4096 * 2
+    w64 = smoe.smoe_workspace_bytes(c, 64)
+    assert w64 < 64 * 8 * 4096 * 2 + (64 * 9) * 4096 * 2 + smoe.smoe_scratch_bytes(c, 64)
     assert smoe.smoe_workspace_bytes(c, 0) > 0
 
 
@@ -71,7 +74,8 @@ def test_argument_errors_before_any_launch():
     assert L.smoe_permute(cp, None, 4, None, 16, 16, 16, 16, None, 256, 1 << 20, None) == smoe.SMOE_ERR_INVALID_ARG
     assert L.smoe_combine(cp, 16, 16, 16, 4, None, 256, 1 << 20, None) == smoe.SMOE_ERR_INVALID_ARG
     assert L.smoe_forward(cp, 16, 4, 16, 16, None, 16, 256, 1 << 30, None) == smoe.SMOE_ERR_INVALID_ARG
-    assert L.smoe_expert_ffn(cp, 16, None, None, 16, 4, 16, 16, 256, 1 << 30, None) == smoe.SMOE_ERR_UNSUPPORTED
+    # neither x_perm nor row_token: nothing to read the routed rows from
+    assert L.smoe_expert_ffn(cp, 16, None, None, 16, 4, 16, 16, 256, 1 << 30, None) == smoe.SMOE_ERR_INVALID_ARG
     assert L.smoe_pack_weights(cp, 16, 16, 16, 16, 16, None, 16, None) == smoe.SMOE_ERR_INVALID_ARG
     # T == 0 is a no-op
     assert L.smoe_forward(cp, None, 0, None, None, None, None, None, 0, None) == 0

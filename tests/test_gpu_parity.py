@@ -130,16 +130,21 @@ def _ffn_sample_rows(offsets, T, k, n_groups=6):
     return sorted(set(int(v) for v in rows))
 
 
+@pytest.mark.parametrize("mode", ["gather", "x_perm"])
 @pytest.mark.parametrize("name", ALL_WORKLOADS)
-def test_expert_ffn_parity(name):
+def test_expert_ffn_parity(name, mode):
+    """gather: routed rows read from x through row_token inside the GEMM; x_perm: from a
+    permuted copy of x built on the host from the oracle's permutation."""
     w, x, _, _, packed = device_inputs(name)
     cfg = cfg_of(w)
     T, k, E = w.T, w.k, w.E
     r = host_route(name)
     _, offsets, _, row_token = oracle.permute(r.idx, E)
     xh = synth.host_x(w)
-    x_perm = torch.from_numpy(xh[row_token].view(np.int16)).cuda().view(torch.bfloat16)
-    y = torch.empty(T * k + T, w.H, dtype=torch.bfloat16, device="cuda")
+    x_perm = None
+    if mode == "x_perm":
+        x_perm = torch.from_numpy(xh[row_token].view(np.int16)).cuda().view(torch.bfloat16)
+    y = torch.full((T * k + T, w.H), float("nan"), dtype=torch.bfloat16, device="cuda")
     ws = _ws(cfg, T)
     smoe.smoe_expert_ffn(cfg, x, x_perm, torch.from_numpy(row_token).cuda(), torch.from_numpy(offsets).cuda(), T,
                          packed, y, ws)
@@ -158,8 +163,9 @@ def test_expert_ffn_parity(name):
         ii = [a for a, _ in items]
         ref[ii] = oracle.swiglu_ffn(x64[[b for _, b in items]], *experts(g))
     assert np.all(np.isfinite(gy[rows]))
-    fro, mx = assert_close(gy[rows], ref, f"{name} expert_ffn")
-    print(f"{name}: expert_ffn rows={len(rows)} rel_fro={fro:.2e} rel_max={mx:.2e}")
+    fro, mx = assert_close(gy[rows], ref, f"{name} expert_ffn ({mode})")
+    assert torch.isfinite(y.float()).all()   # every row written
+    print(f"{name}: expert_ffn ({mode}) rows={len(rows)} rel_fro={fro:.2e} rel_max={mx:.2e}")
 
 
 # ------------------------------------------------------------------------------ combine
@@ -275,8 +281,12 @@ def test_forward_is_deterministic_and_matches_per_call_chain():
     out3 = torch.empty(T, w.H, dtype=torch.bfloat16, device="cuda")
     smoe.smoe_route(cfg, x, T, wr, bias, idx, wt, None, ws)
     smoe.smoe_permute(cfg, idx, T, x, counts, offsets, perm_row, row_token, x_perm, ws)
-    smoe.smoe_expert_ffn(cfg, x, x_perm, row_token, offsets, T, packed, y, ws)
+    smoe.smoe_expert_ffn(cfg, x, None, row_token, offsets, T, packed, y, ws)
     smoe.smoe_combine(cfg, y, perm_row, wt, T, out3, ws)
+    # the permuted-copy path gives the same bits
+    y2 = torch.empty_like(y)
+    smoe.smoe_expert_ffn(cfg, x, x_perm, row_token, offsets, T, packed, y2, ws)
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
     assert smoe.smoe_get_device_error(ws) == 0
     assert torch.equal(out1.view(torch.int16), out3.view(torch.int16))
 
