@@ -47,7 +47,10 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
 constexpr int kNumTiles = 5;     // token tiles 16, 32, 64, 128, 256
-constexpr int kMaxStages = 24;
+#ifndef SMOE_MAX_STAGES
+#define SMOE_MAX_STAGES 24       // cap on the pipeline depth (a tuning constant, <= 32)
+#endif
+constexpr int kMaxStages = SMOE_MAX_STAGES;
 
 struct GemmMaps {
     CUtensorMap w;                  // weights [rows][K]: box {BK, 256 (gate/up) or 128 (down)}
@@ -230,7 +233,10 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     const uint32_t tmem_base = *tmem_slot;
     const int total = prefix[E + 1];
 
-    if (warp == 0) {
+    // gather mode (row_token set) uses all 32 producer lanes; otherwise lane 0 alone, so the
+    // stage refill path carries no warp-wide synchronisation
+    const unsigned pmask = (p.row_token != nullptr) ? 0xFFFFFFFFu : 1u;
+    if (warp == 0 && ((pmask >> lane) & 1u)) {
         // ---------------------------------------------------------------- TMA producer (warp 0)
         // Lane 0 waits for a free stage, arms its barrier and loads the weight tile. Activation
         // rows come either as one tile (contiguous rows) or, for routed groups in gather mode,
@@ -265,7 +271,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             }
             for (int kb = 0; kb < KB; ++kb) {
                 if (lane == 0) ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag, true);
-                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                ok = __shfl_sync(pmask, ok, 0);
                 if (!ok) break;
                 const uint32_t fb = smem_u32(&full[stage]);
                 uint8_t* a_s = tiles + (size_t)stage * STAGE_B;
@@ -275,7 +281,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                     tma_load_2d(smem_u32(a_s), &maps.w, kb * BK, a_row, fb, pol_w);
                     if (!gather) tma_load_2d(smem_u32(a_s + C::A_BYTES), bm, b_k * BK, b_row, fb, pol_a);
                 }
-                __syncwarp();
+                __syncwarp(pmask);
                 if (gather) {
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
@@ -294,7 +300,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         if (lane == 0)
             for (int s = 0; s < S; ++s)
                 if ((armed >> s) & 1u) mbar_wait(smem_u32(&full[s]), (armed_par >> s) & 1u, p.err, abort_flag, false);
-        __syncwarp();
+        __syncwarp(pmask);
     } else if (warp == 1 && lane == 0) {
         // ---------------------------------------------------------------- MMA issuer
         const uint32_t idesc0 = idesc_bf16_f32(128, 0);

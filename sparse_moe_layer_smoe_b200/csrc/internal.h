@@ -11,14 +11,13 @@ namespace smoe {
 
 constexpr size_t kAlign = 256;
 constexpr int kPermuteTokensPerBlock = 256;
-constexpr int kRouterKChunk = 32;
 
 inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
 
 // Router plan for T tokens. CUDA cores: tokens per CTA, experts per CTA, K splits. Tensor cores
 // (tc, large T): W_r split into three bf16 pieces in the workspace, token tile nt.
 struct RouterPlan {
-    int tm, te, splits;
+    int tm, te, kc, splits;
     bool tc;
     int nt, e_pad;
     size_t scratch_bytes;   // partial logits (+ the split weights when tc)

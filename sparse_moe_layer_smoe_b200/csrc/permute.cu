@@ -13,6 +13,7 @@
 //                          lane bitmasks in shared memory (a token picks an expert at most
 //                          once), warp prefix over the block, block base from the scan
 //   gather_rows_kernel     x_perm[r] = x[row_token[r]], one warp per row, 16-byte accesses
+//   permute_small_kernel   T <= 1024: histogram, scan and scatter in one CTA (same results)
 // An expert id outside [0, E) or repeated within a token is skipped (perm_row = -1) and
 // recorded as SMOE_ERR_DEVICE.
 #include "common.cuh"
@@ -141,6 +142,84 @@ __global__ void __launch_bounds__(TB) permute_scatter_kernel(const int32_t* __re
     (void)err;
 }
 
+// The whole permutation in one CTA of up to 1024 threads (one token per thread), for T <= 1024:
+// the same histogram, scan and stable rank as the three kernels above, kept in shared memory.
+// Outputs are identical to the multi-block path.
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallWarps = kSmallThreads / 32;
+
+__global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(const int32_t* __restrict__ idx, int T, int k,
+                                                                      int E, int32_t* __restrict__ counts,
+                                                                      int32_t* __restrict__ offsets,
+                                                                      int32_t* __restrict__ perm_row,
+                                                                      int32_t* __restrict__ row_token, int32_t* err) {
+    extern __shared__ uint32_t smem[];
+    uint32_t* wmask = smem;                                                  // [warps][E]
+    int32_t* wbase = reinterpret_cast<int32_t*>(smem + kSmallWarps * E);     // [warps][E]
+    int32_t* offs = wbase + kSmallWarps * E;                                 // [E + 1]
+    __shared__ int32_t warp_tot[32];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < kSmallWarps * E; i += kSmallThreads) wmask[i] = 0u;
+    __syncthreads();
+    const int t = threadIdx.x;
+    if (t < T) {
+        for (int j = 0; j < k; ++j)
+            if (entry_valid(idx, t, j, k, E, err)) atomicOr(&wmask[w * E + idx[(size_t)t * k + j]], 1u << lane);
+    }
+    __syncthreads();
+    // per-expert warp prefix and totals; then an exclusive scan over experts (E <= 1024)
+    int32_t cnt = 0;
+    const int e = threadIdx.x;
+    if (e < E) {
+        for (int q = 0; q < kSmallWarps; ++q) {
+            wbase[q * E + e] = cnt;
+            cnt += __popc(wmask[q * E + e]);
+        }
+        counts[e] = cnt;
+    }
+    int32_t v = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int32_t n = __shfl_up_sync(0xFFFFFFFFu, v, off);
+        if (lane >= off) v += n;
+    }
+    if (lane == 31) warp_tot[w] = v;
+    __syncthreads();
+    if (w == 0) {
+        int32_t tv = warp_tot[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int32_t n = __shfl_up_sync(0xFFFFFFFFu, tv, off);
+            if (lane >= off) tv += n;
+        }
+        warp_tot[lane] = tv;
+    }
+    __syncthreads();
+    const int32_t incl = v + (w > 0 ? warp_tot[w - 1] : 0);
+    if (e < E) {
+        offs[e] = incl - cnt;
+        offsets[e] = incl - cnt;
+    }
+    if (e == E - 1) offsets[E] = incl;
+    __syncthreads();
+    if (t < T) {
+        const uint32_t below = (1u << lane) - 1u;
+        for (int j = 0; j < k; ++j) {
+            const int ex = idx[(size_t)t * k + j];
+            bool ok = (ex >= 0 && ex < E);
+            for (int q = 0; ok && q < j; ++q) ok = idx[(size_t)t * k + q] != ex;
+            int32_t row = -1;
+            if (ok) {
+                row = offs[ex] + wbase[w * E + ex] + __popc(wmask[w * E + ex] & below);
+                row_token[row] = t;
+            }
+            perm_row[(size_t)t * k + j] = row;
+        }
+    }
+}
+
+size_t permute_small_smem(int E) { return (2 * (size_t)kSmallWarps * E + E + 1) * sizeof(int32_t); }
+
 // x_perm[r] = x[row_token[r]] for r < offsets[E]; one warp per row.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,
                                                           const int32_t* __restrict__ row_token,
@@ -168,28 +247,44 @@ cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int6
                            uint16_t* x_perm, int32_t* hist, int32_t* base, int32_t* err, cudaStream_t s) {
     const int E = c.n_experts, k = c.top_k;
     const int nblk = (int)((T + TB - 1) / TB);
-    {
-        LaunchTimer lt(K_PERMUTE_HIST, s);
-        permute_hist_kernel<<<nblk, TB, E * sizeof(int32_t), s>>>(topk_idx, (int)T, k, E, hist, err);
-    }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    {
-        LaunchTimer lt(K_PERMUTE_SCAN, s);
-        permute_scan_kernel<<<1, 1024, 0, s>>>(hist, nblk, E, base, counts, offsets);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const size_t sm = 2 * WARPS * E * sizeof(uint32_t);
-    if (sm > 48 * 1024) {
-        e = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        if (e != cudaSuccess) return e;
-    }
-    {
-        LaunchTimer lt(K_PERMUTE_SCATTER, s);
-        permute_scatter_kernel<<<nblk, TB, sm, s>>>(topk_idx, (int)T, k, E, base, offsets, perm_row, row_token, err);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    cudaError_t e;
     int n = 3;
+    const size_t small_sm = permute_small_smem(E);
+    if (T <= kSmallThreads && small_sm <= 200 * 1024) {
+        if (small_sm > 48 * 1024) {
+            e = cudaFuncSetAttribute(permute_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)small_sm);
+            if (e != cudaSuccess) return e;
+        }
+        {
+            LaunchTimer lt(K_PERMUTE_SCATTER, s);
+            permute_small_kernel<<<1, kSmallThreads, small_sm, s>>>(topk_idx, (int)T, k, E, counts, offsets, perm_row,
+                                                                    row_token, err);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        n = 1;
+    } else {
+        {
+            LaunchTimer lt(K_PERMUTE_HIST, s);
+            permute_hist_kernel<<<nblk, TB, E * sizeof(int32_t), s>>>(topk_idx, (int)T, k, E, hist, err);
+        }
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        {
+            LaunchTimer lt(K_PERMUTE_SCAN, s);
+            permute_scan_kernel<<<1, 1024, 0, s>>>(hist, nblk, E, base, counts, offsets);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const size_t sm = 2 * WARPS * E * sizeof(uint32_t);
+        if (sm > 48 * 1024) {
+            e = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+            if (e != cudaSuccess) return e;
+        }
+        {
+            LaunchTimer lt(K_PERMUTE_SCATTER, s);
+            permute_scatter_kernel<<<nblk, TB, sm, s>>>(topk_idx, (int)T, k, E, base, offsets, perm_row, row_token, err);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     if (x != nullptr && x_perm != nullptr) {
         const int64_t rows = T * k;
         int64_t blocks = (rows + 7) / 8;

@@ -25,27 +25,29 @@ namespace smoe {
 
 namespace {
 
-template <int TM, int TE, int RM, int RE>
+template <int TM, int TE, int RM, int RE, int KC_>
 struct RouterTile {
     static constexpr int TX = TE / RE;          // threads along experts
     static constexpr int TY = TM / RM;          // threads along tokens
     static constexpr int THREADS = TX * TY;
-    static constexpr int KC = kRouterKChunk;    // K elements per stage
+    static constexpr int KC = KC_;              // K elements per stage
     static constexpr int XCHUNKS = TM * KC / 8; // 16-byte chunks of x per stage
     static constexpr int WCHUNKS = TE * KC / 4; // 16-byte chunks of W_r per stage
     static constexpr int XPT = (XCHUNKS + THREADS - 1) / THREADS;
     static constexpr int WPT = (WCHUNKS + THREADS - 1) / THREADS;
 };
 
-template <int TM, int TE, int RM, int RE>
-__global__ void __launch_bounds__(RouterTile<TM, TE, RM, RE>::THREADS)
+template <int TM, int TE, int RM, int RE, int KC_>
+__global__ void __launch_bounds__(RouterTile<TM, TE, RM, RE, KC_>::THREADS)
 router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr, float* __restrict__ part,
                      int T, int E, int H, int k_len) {
-    using P = RouterTile<TM, TE, RM, RE>;
+    using P = RouterTile<TM, TE, RM, RE, KC_>;
     constexpr int KC = P::KC;
-    // +1 padding: the transposing stores below hit 32 distinct banks
-    __shared__ float xs[2][KC][TM + 1];
-    __shared__ float ws[2][KC][TE + 1];
+    // two stages of x [KC][TM+1] and W_r [KC][TE+1]; +1 padding: the transposing stores below
+    // hit 32 distinct banks
+    extern __shared__ float rsm[];
+    float (*xs)[KC][TM + 1] = reinterpret_cast<float (*)[KC][TM + 1]>(rsm);
+    float (*ws)[KC][TE + 1] = reinterpret_cast<float (*)[KC][TE + 1]>(rsm + 2 * KC * (TM + 1));
 
     const int tid = threadIdx.x;
     const int tx = tid % P::TX, ty = tid / P::TX;
@@ -172,8 +174,17 @@ router_topk_kernel(const float* __restrict__ part, int splits, const float* __re
         S[i] = 0.f;
         B[i] = -INFINITY;
         if (e < E) {
+            // partial sums added in split order 0, 1, 2, ... (four loads in flight at a time)
+            const float* pe = part + (size_t)t * E + e;
+            const size_t stride = (size_t)T * E;
             float l = 0.f;
-            for (int s = 0; s < splits; ++s) l += part[((size_t)s * T + t) * E + e];
+            int s = 0;
+            for (; s + 4 <= splits; s += 4) {
+                const float a = pe[s * stride], b = pe[(s + 1) * stride], c = pe[(s + 2) * stride],
+                            d = pe[(s + 3) * stride];
+                l = (((l + a) + b) + c) + d;
+            }
+            for (; s < splits; ++s) l += pe[s * stride];
             L[i] = l;
             if (logits_out) logits_out[(size_t)t * E + e] = l;
             const float sg = 1.0f / (1.0f + expf(-l));
@@ -261,14 +272,20 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
     }
 }
 
-template <int TM, int TE, int RM, int RE>
+template <int TM, int TE, int RM, int RE, int KC>
 cudaError_t launch_logits(const uint16_t* x, int64_t T, const float* wr, int E, int H, int splits, float* part,
                           cudaStream_t s) {
-    using P = RouterTile<TM, TE, RM, RE>;
+    using P = RouterTile<TM, TE, RM, RE, KC>;
     dim3 grid((unsigned)((T + TM - 1) / TM), (unsigned)((E + TE - 1) / TE), (unsigned)splits);
+    const int smem = (int)(2 * KC * (TM + 1 + TE + 1) * sizeof(float));
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(router_logits_kernel<TM, TE, RM, RE, KC>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+    }
     {
         LaunchTimer lt(K_ROUTER_LOGITS, s);
-        router_logits_kernel<TM, TE, RM, RE><<<grid, P::THREADS, 0, s>>>(x, wr, part, (int)T, E, H, H / splits);
+        router_logits_kernel<TM, TE, RM, RE, KC><<<grid, P::THREADS, smem, s>>>(x, wr, part, (int)T, E, H, H / splits);
     }
     return cudaGetLastError();
 }
@@ -307,12 +324,14 @@ RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms, bool allo
     if (T >= 512) {
         p.tm = 64;
         p.te = (E % 96 == 0) ? 96 : 64;
+        p.kc = 32;
     } else {
         p.tm = 16;
         p.te = 32;
+        p.kc = 128;   // few, long K slices: each CTA waits on 4 load rounds, not 16
     }
     const int64_t base = ((T + p.tm - 1) / p.tm) * ((E + p.te - 1) / p.te);
-    const int chunks = c.hidden / kRouterKChunk;
+    const int chunks = c.hidden / p.kc;
     int splits = 1;
     while (splits * 2 <= 16 && chunks % (splits * 2) == 0 && base * splits * 2 <= 2 * (int64_t)num_sms) splits *= 2;
     p.splits = splits;
@@ -339,11 +358,11 @@ cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, c
         e = launch_router_gemm(x, T, H, w_split, p.e_pad, E, partials, p.nt, num_sms, s);
         n = 3;
     } else if (p.tm == 64 && p.te == 96) {
-        e = launch_logits<64, 96, 4, 6>(x, T, wr, E, H, p.splits, partials, s);
+        e = launch_logits<64, 96, 4, 6, 32>(x, T, wr, E, H, p.splits, partials, s);
     } else if (p.tm == 64) {
-        e = launch_logits<64, 64, 4, 4>(x, T, wr, E, H, p.splits, partials, s);
+        e = launch_logits<64, 64, 4, 4, 32>(x, T, wr, E, H, p.splits, partials, s);
     } else {
-        e = launch_logits<16, 32, 2, 2>(x, T, wr, E, H, p.splits, partials, s);
+        e = launch_logits<16, 32, 2, 2, 128>(x, T, wr, E, H, p.splits, partials, s);
     }
     if (e != cudaSuccess) return e;
     const int npl = (E + 31) / 32;
