@@ -51,6 +51,10 @@ constexpr int kNumTiles = 5;     // token tiles 16, 32, 64, 128, 256
 #define SMOE_MAX_STAGES 24       // cap on the pipeline depth (a tuning constant, <= 32)
 #endif
 constexpr int kMaxStages = SMOE_MAX_STAGES;
+#ifndef SMOE_PAIR_MIN_TILE
+#define SMOE_PAIR_MIN_TILE 64    // CTA pairs for launches whose largest token tile is at least this
+#endif
+constexpr int kPairMinTile = SMOE_PAIR_MIN_TILE;
 
 struct GemmMaps {
     CUtensorMap w;                  // weights [rows][K]: box {BK, 256 (gate/up) or 128 (down)}
@@ -134,6 +138,48 @@ __device__ __forceinline__ Unit decode_unit(int u, const int32_t* prefix, const 
     const int nblk = (rows + nt - 1) / nt;
     const int local = u - prefix[g];
     return Unit{g, local / nblk, local % nblk, nt};
+}
+
+// Epilogue, part 1: drain this thread's accumulator row (one output feature, up to 256 token
+// columns) into registers as packed bf16 pairs: SiLU(gate) * up for gate/up, the plain value for
+// down. 32-column TMEM loads, one wait each. nch = number of 32-column chunks holding valid tokens.
+template <bool DUAL>
+__device__ __forceinline__ void epi_load(uint32_t t_row, int nt_max, int nch, uint32_t (&hv)[128]) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        if (c < nch) {
+            uint32_t a[32], b[32];
+            if (DUAL)
+                tmem_ld2_x32_wait(t_row + 32 * c, t_row + nt_max + 32 * c, a, b);
+            else
+                tmem_ld_x32_wait(t_row + 32 * c, a);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                float v0 = __uint_as_float(a[2 * j]), v1 = __uint_as_float(a[2 * j + 1]);
+                if (DUAL) {
+                    v0 = silu_mul(v0, __uint_as_float(b[2 * j]));
+                    v1 = silu_mul(v1, __uint_as_float(b[2 * j + 1]));
+                }
+                hv[16 * c + j] = (uint32_t)float_to_bf16_bits(v0) | ((uint32_t)float_to_bf16_bits(v1) << 16);
+            }
+        }
+    }
+}
+
+// Epilogue, part 2: store the valid token columns of this thread's feature (after the accumulator
+// has been handed back to the MMA thread).
+__device__ __forceinline__ void epi_store(const uint32_t (&hv)[128], int nch, int nvalid, uint16_t* out, size_t dst0,
+                                          int ld) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        if (c < nch) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (32 * c + j < nvalid)
+                    out[dst0 + (size_t)(32 * c + j) * ld] = (uint16_t)((j & 1) ? (hv[16 * c + j / 2] >> 16)
+                                                                               : (hv[16 * c + j / 2] & 0xFFFFu));
+        }
+    }
 }
 
 template <int MODE, int BK>
@@ -359,29 +405,24 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             const int f = w.mb * 128 + row;
             const bool keep = f < p.out_valid;
             const size_t dst0 = (size_t)out_base * p.out_ld + f;
-            for (int c0 = 0; c0 < nvalid; c0 += 16) {
-                uint32_t g16[16], u16[16];
-                if (DUAL)
-                    tmem_ld2_x16_wait(t_row + c0, t_row + p.nt_max + c0, g16, u16);
-                else
+            if (MODE == MODE_ROUTER) {
+                for (int c0 = 0; c0 < nvalid; c0 += 16) {
+                    uint32_t g16[16];
                     tmem_ld_x16_wait(t_row + c0, g16);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    if (c0 + j < nvalid && keep) {
-                        const float gv = __uint_as_float(g16[j]);
-                        const size_t o = dst0 + (size_t)(c0 + j) * p.out_ld;
-                        if (MODE == MODE_ROUTER) {
-                            p.out_f32[o] = gv;
-                        } else {
-                            float v = gv;
-                            if (DUAL) v = (gv / (1.0f + expf(-gv))) * __uint_as_float(u16[j]);
-                            p.out[o] = float_to_bf16_bits(v);
-                        }
-                    }
+                    for (int j = 0; j < 16; ++j)
+                        if (c0 + j < nvalid && keep) p.out_f32[dst0 + (size_t)(c0 + j) * p.out_ld] = __uint_as_float(g16[j]);
                 }
+                tc_fence_before();
+                mbar_arrive(smem_u32(&tempty[acc]));
+            } else {
+                const int nch = (nvalid + 31) / 32;
+                uint32_t hv[128];
+                epi_load<DUAL>(t_row, p.nt_max, nch, hv);
+                tc_fence_before();
+                mbar_arrive(smem_u32(&tempty[acc]));   // accumulator free before the stores
+                epi_store(hv, nch, nvalid, p.out, dst0, p.out_ld);
             }
-            tc_fence_before();
-            mbar_arrive(smem_u32(&tempty[acc]));
             if (NACC == 2) {
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
@@ -396,6 +437,241 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// CTA-pair variant (tcgen05 cta_group::2) for large token tiles.
+//
+// A pair of CTAs on two SMs computes one unit of 256 output features x nt tokens: each CTA
+// holds the weight rows of its 128 features (for gate/up: 128 gate + 128 up rows) and half of
+// the token rows (nt/2); one 256-row MMA issued by the first CTA reads both CTAs' shared memory
+// and accumulates into both CTAs' TMEM (128 rows each). Per SM this moves 25-30% fewer operand
+// bytes through shared memory per MMA than the single-CTA kernel, whose token tile every SM
+// loads in full. Work unit = (group, 256-feature block, token tile); pair p takes units p,
+// p + pairs, ...
+//
+// Signals: both CTAs' loads complete on the first CTA's stage barrier (it arms the expected
+// bytes of both); the first CTA's MMA thread commits stage-free and accumulator-ready to each
+// CTA's barrier; both CTAs' epilogue warps arrive on the first CTA's accumulator-free barrier.
+// A cluster barrier before teardown keeps each CTA's shared memory and TMEM alive until the
+// pair's MMAs are done.
+// ------------------------------------------------------------------------------------------
+template <int MODE, int BK>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
+    using C = GemmCfg<MODE, BK>;
+    constexpr bool DUAL = C::DUAL;
+    extern __shared__ uint8_t smem_raw[];
+    const int S = p.stages;
+    const int STAGE_B = C::A_BYTES + (p.nt_max / 2) * BK * 2;
+    const int ACC_COLS = DUAL ? 2 * p.nt_max : p.nt_max;
+    const int NACC = (2 * ACC_COLS <= kTmemCols) ? 2 : 1;
+    uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(tiles + (size_t)S * STAGE_B);
+    uint64_t* empty = full + S;
+    uint64_t* tfull = empty + S;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int32_t* prefix = reinterpret_cast<int32_t*>(tmem_slot + 4);   // [E+2]
+    int32_t* offs = prefix + (p.E + 2);                              // [E+1]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int E = p.E;
+    const int MB = p.n_out / 128;       // 128-row blocks of a group's weights
+    const int MBP = p.n_out / 256;      // 256-feature blocks handled by a pair
+    const int KB = p.K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), 8);   // 4 epilogue warps x 2 CTAs
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish_pair();
+    }
+    if (warp == 1 && lane == 0) {
+        tma_prefetch_desc(&maps.w);
+        for (int i = 0; i < kNumTiles; ++i)
+            if ((16 << i) <= p.nt_max) {
+                tma_prefetch_desc(&maps.act[i]);
+                tma_prefetch_desc(&maps.sh[i]);
+            }
+    }
+    if (warp == 2) {
+        bool bad = false;
+        for (int i = lane; i <= E; i += 32) {
+            int v = (p.offsets != nullptr) ? p.offsets[i] : 0;
+            if (v < 0 || v > p.routed_rows) { bad = true; v = 0; }
+            offs[i] = v;
+        }
+        __syncwarp();
+        for (int i = lane; i < E; i += 32)
+            if (offs[i + 1] < offs[i]) bad = true;
+        if (__any_sync(0xFFFFFFFFu, bad)) {
+            for (int i = lane; i <= E; i += 32) offs[i] = 0;
+            if (lane == 0) record_error(p.err, SMOE_ERR_DEVICE);
+        }
+        __syncwarp();
+        const int ngroups = E + 1;
+        const int chunk = (ngroups + 31) / 32;
+        const int g0 = min(lane * chunk, ngroups), g1 = min(g0 + chunk, ngroups);
+        auto units_of = [&](int g) {
+            const int rows = group_rows(g, E, p.T, offs);
+            const int nt = group_tile(rows, p.nt_max);
+            return ((rows + nt - 1) / nt) * MBP;
+        };
+        int local = 0;
+        for (int g = g0; g < g1; ++g) local += units_of(g);
+        int incl = local;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int n = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+            if (lane >= off) incl += n;
+        }
+        int run = incl - local;
+        for (int g = g0; g < g1; ++g) {
+            prefix[g] = run;
+            run += units_of(g);
+        }
+        if (lane == 31) prefix[E + 1] = incl;
+    }
+    tc_fence_before();
+    cluster_sync();   // barrier inits and TMEM allocation visible to both CTAs
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = prefix[E + 1];
+
+    if (warp == 0 && lane == 0) {
+        // ---------------------------------------------------------------- TMA producer (both CTAs)
+        const uint64_t pol_w = l2_policy_evict_first();
+        const uint64_t pol_a = l2_policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0, armed = 0, armed_par = 0;
+        bool ok = true;
+        for (int u = pair; ok && u < total; u += npairs) {
+            const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);   // w.mb = 256-feature block
+            const int a_row = DUAL ? (w.g * MB + 2 * w.mb + (int)rank) * 256 : w.g * p.n_out + w.mb * 256 + (int)rank * 128;
+            const int half = w.nt / 2;
+            const int b_row = (w.g < E ? offs[w.g] : p.shared_in_row) + w.nb * w.nt + (int)rank * half;
+            const int ti = tile_index(w.nt);
+            const CUtensorMap* bm = (w.g < E) ? &maps.act[ti] : &maps.sh[ti];
+            const uint32_t tx = (uint32_t)(2 * (C::A_BYTES + half * BK * 2));
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag, true)) { ok = false; break; }
+                const uint32_t fb_local = smem_u32(&full[stage]);
+                const uint32_t fb_leader = mapa_shared(fb_local, 0);
+                if (rank == 0) mbar_arrive_expect_tx(fb_local, tx);
+                uint8_t* a_s = tiles + (size_t)stage * STAGE_B;
+                tma_load_2d_pair(smem_u32(a_s), &maps.w, kb * BK, a_row, fb_leader, pol_w);
+                tma_load_2d_pair(smem_u32(a_s + C::A_BYTES), bm, kb * BK, b_row, fb_leader, pol_a);
+                armed |= 1u << stage;
+                armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+                if (++stage == S) { stage = 0; phase ^= 1u; }
+            }
+        }
+        if (rank == 0) {
+            // both CTAs' bytes of every armed stage are counted here: wait for them to land
+            for (int s = 0; s < S; ++s)
+                if ((armed >> s) & 1u)
+                    mbar_wait(smem_u32(&full[s]), (armed_par >> s) & 1u, p.err, abort_flag, false);
+        }
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+        // ---------------------------------------------------------------- MMA issuer (first CTA)
+        const uint32_t idesc0 = idesc_bf16_f32(256, 0);
+        int stage = 0, acc = 0;
+        uint32_t phase = 0, acc_phase = 0;
+        bool ok = true;
+        for (int u = pair; ok && u < total; u += npairs) {
+            const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
+            const uint32_t idesc = idesc0 | ((uint32_t)(w.nt >> 3) << 17);
+            if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, p.err, abort_flag, true)) break;
+            tc_fence_after();
+            const uint32_t d = tmem_base + (uint32_t)(acc * ACC_COLS);
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(smem_u32(&full[stage]), phase, p.err, abort_flag, true)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a_s = smem_u32(tiles + (size_t)stage * STAGE_B);
+                const uint32_t b_s = a_s + C::A_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+                    const uint64_t bdesc = smem_desc_kmajor<C::SW>(b_s + kk * 32);
+                    umma_f16_ss_pair(d, smem_desc_kmajor<C::SW>(a_s + kk * 32), bdesc, idesc, accum);
+                    if (DUAL)
+                        umma_f16_ss_pair(d + p.nt_max, smem_desc_kmajor<C::SW>(a_s + C::UP_OFFSET + kk * 32), bdesc,
+                                         idesc, accum);
+                }
+                const uint32_t eb = smem_u32(&empty[stage]);
+                umma_commit_pair(mapa_shared(eb, 0));
+                umma_commit_pair(mapa_shared(eb, 1));
+                if (++stage == S) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            const uint32_t tb = smem_u32(&tfull[acc]);
+            umma_commit_pair(mapa_shared(tb, 0));
+            umma_commit_pair(mapa_shared(tb, 1));
+            if (NACC == 2) {
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            } else {
+                acc_phase ^= 1u;
+            }
+        }
+        umma_commit_pair(mapa_shared(smem_u32(drain), 0));
+        mbar_wait(smem_u32(drain), 0u, p.err, abort_flag, false);
+    } else if (warp >= 2) {
+        // ---------------------------------------------------------------- epilogue (both CTAs)
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = pair; u < total; u += npairs) {
+            const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
+            const int rows = group_rows(w.g, E, p.T, offs);
+            const int out_base = (w.g < E ? offs[w.g] : p.shared_out_row) + w.nb * w.nt;
+            const int nvalid = min(w.nt, rows - w.nb * w.nt);
+            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.err, abort_flag, true)) break;
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+            const int f = w.mb * 256 + (int)rank * 128 + row;
+            const size_t dst0 = (size_t)out_base * p.out_ld + f;
+            const int nch = (nvalid + 31) / 32;
+            uint32_t hv[128];
+            epi_load<DUAL>(t_row, p.nt_max, nch, hv);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));   // accumulator free
+            epi_store(hv, nch, nvalid, p.out, dst0, p.out_ld);
+            if (NACC == 2) {
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            } else {
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) __nanosleep(100000);   // give loads still in flight after a timeout time to land
+    cluster_sync();   // the peer's shared memory and TMEM stay alive until the pair's MMAs are done
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
     }
 }
 
@@ -481,6 +757,53 @@ cudaError_t run_gemm(const GemmMaps& maps, GemmParams p, int grid, cudaStream_t 
     return cudaGetLastError();
 }
 
+// Activation maps for CTA pairs: each CTA loads half of a token tile (box rows 8 << i).
+bool make_half_act_maps(CUtensorMap* maps, const void* base, uint64_t rows, uint64_t cols, int nt_max, int bk) {
+    for (int i = 0; i < kNumTiles; ++i) {
+        const int nt = 16 << i;
+        if (nt <= nt_max) {
+            if (!make_map(&maps[i], base, rows, cols, nt / 2, bk)) return false;
+        } else {
+            maps[i] = maps[i - 1];
+        }
+    }
+    return true;
+}
+
+template <int MODE>
+cudaError_t run_gemm_pair(const GemmMaps& maps, GemmParams p, int num_sms, cudaStream_t s) {
+    constexpr int BK = SMOE_GEMM_BK;
+    constexpr bool DUAL = MODE == MODE_GATEUP;
+    const int sb = (DUAL ? 256 : 128) * BK * 2 + (p.nt_max / 2) * BK * 2;
+    const size_t fixed = gemm_smem_bytes(0, sb, p.E) + 2 * sizeof(uint64_t) * kMaxStages;
+    int stages = (int)((max_dynamic_smem() - fixed) / sb);
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages < 2) return cudaErrorInvalidConfiguration;
+    p.stages = stages;
+    const size_t smem = gemm_smem_bytes(stages, sb, p.E);
+    auto kern = expert_gemm_pair_kernel<MODE, BK>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // pairs resident at once (a GPC with an odd number of free SMs cannot host a pair there)
+    static int max_clusters[3] = {0, 0, 0};
+    if (max_clusters[MODE] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(num_sms & ~1);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+        if (e != cudaSuccess) return e;
+        max_clusters[MODE] = n > 0 ? n : 1;
+    }
+    const int pairs = std::min(num_sms / 2, max_clusters[MODE]);
+    {
+        LaunchTimer lt(MODE == MODE_GATEUP ? K_EXPERT_GATEUP : K_EXPERT_DOWN, s);
+        kern<<<2 * pairs, kThreads, smem, s>>>(maps, p);
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 // Largest token tile of a launch: the smallest power of two >= 1.25 x the mean rows per routed
@@ -509,24 +832,28 @@ cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const u
 
     GemmMaps m1, m2;
     const bool gather = x_perm == nullptr;
-    bool ok_act = gather ? make_map(&m1.act[0], x, (uint64_t)T, H, 1, BK)
-                         : make_act_maps(m1.act, x_perm, (uint64_t)routed, H, nt, BK);
+    // CTA pairs for large token tiles (each pair handles 256 output features)
+    const bool pairs = !gather && nt >= kPairMinTile && I % 256 == 0 && H % 256 == 0;
+    auto act_maps = [&](CUtensorMap* maps, const void* base, uint64_t rows, uint64_t cols) {
+        return pairs ? make_half_act_maps(maps, base, rows, cols, nt, BK) : make_act_maps(maps, base, rows, cols, nt, BK);
+    };
+    bool ok_act = gather ? make_map(&m1.act[0], x, (uint64_t)T, H, 1, BK) : act_maps(m1.act, x_perm, (uint64_t)routed, H);
     if (gather)
         for (int i = 1; i < kNumTiles; ++i) m1.act[i] = m1.act[0];
     if (!ok_act || !make_map(&m1.w, wgu, (uint64_t)(E + 1) * 2 * I, H, 256, BK) ||
-        !make_act_maps(m1.sh, x, (uint64_t)T, H, nt, BK) ||
+        !act_maps(m1.sh, x, (uint64_t)T, H) ||
         !make_map(&m2.w, wdn, (uint64_t)(E + 1) * H, I, 128, BK) ||
-        !make_act_maps(m2.act, h, (uint64_t)(routed + T), I, nt, BK))
+        !act_maps(m2.act, h, (uint64_t)(routed + T), I))
         return cudaErrorNotSupported;
     for (int i = 0; i < kNumTiles; ++i) m2.sh[i] = m2.act[i];
 
     GemmParams p1{offsets, E, (int)T, (int)routed, H, I, 0, (int)routed, nt, 0, 0, I, I, gather ? row_token : nullptr,
                   h, nullptr, err};
-    cudaError_t e = run_gemm<MODE_GATEUP>(m1, p1, num_sms, s);
+    cudaError_t e = pairs ? run_gemm_pair<MODE_GATEUP>(m1, p1, num_sms, s) : run_gemm<MODE_GATEUP>(m1, p1, num_sms, s);
     if (e != cudaSuccess) return e;
     GemmParams p2{offsets, E, (int)T, (int)routed, I, H, (int)routed, (int)routed, nt, 0, 0, H, H, nullptr, y, nullptr,
                   err};
-    e = run_gemm<MODE_DOWN>(m2, p2, num_sms, s);
+    e = pairs ? run_gemm_pair<MODE_DOWN>(m2, p2, num_sms, s) : run_gemm<MODE_DOWN>(m2, p2, num_sms, s);
     if (e == cudaSuccess) launches_add(2);
     return e;
 }
