@@ -347,7 +347,7 @@ def run_ours(args):
         launches, tot = ktimes[dom]
         avg_s = tot / launches / 1e3
         intensity = kern_flops[dom] / kern_bytes[dom]
-        ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
         if intensity < ridge:
             ach = kern_bytes[dom] / avg_s / 1e9
             roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",

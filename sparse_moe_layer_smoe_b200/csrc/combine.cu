@@ -48,11 +48,23 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-        for (int j = 0; j < k; ++j) {
-            const int r = rows[j];
-            if (r >= 0) fma8(acc, ws[j], y4[(size_t)r * vec + c]);
+        const uint4 shared_row = y4[(size_t)(nrouted + t) * vec + c];
+        if (k <= 8) {
+            // all rows' vectors in flight first, then the FMAs in slot order
+            uint4 v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j < k && rows[j] >= 0) v[j] = y4[(size_t)rows[j] * vec + c];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j < k && rows[j] >= 0) fma8(acc, ws[j], v[j]);
+        } else {
+            for (int j = 0; j < k; ++j) {
+                const int r = rows[j];
+                if (r >= 0) fma8(acc, ws[j], y4[(size_t)r * vec + c]);
+            }
         }
-        fma8(acc, 1.0f, y4[(size_t)(nrouted + t) * vec + c]);
+        fma8(acc, 1.0f, shared_row);
         uint4 o;
         uint32_t* ou = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll

@@ -77,6 +77,8 @@ struct GemmParams {
     int out_ld;               // leading dimension of the output rows
     int out_valid;            // output features stored: f < out_valid
     const int32_t* row_token; // gather mode (routed groups read x rows by token), else nullptr
+    int ksplit;               // K split into this many equal ranges, one unit each (router pieces)
+    size_t split_stride;      // elements between the partial outputs of consecutive K ranges
     uint16_t* out;            // [*, out_ld] bf16 (gate/up, down)
     float* out_f32;           // [*, out_ld] fp32 (router)
     int32_t* err;
@@ -206,7 +208,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
     const int MB = p.n_out / 128;
-    const int KB = p.K / BK;
+    const int KB = p.K / BK / p.ksplit;   // k-blocks of one unit
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -256,7 +258,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         auto units_of = [&](int g) {
             const int rows = group_rows(g, E, p.T, offs);
             const int nt = group_tile(rows, p.nt_max);
-            return ((rows + nt - 1) / nt) * MB;
+            return ((rows + nt - 1) / nt) * MB * p.ksplit;
         };
         int local = 0;
         for (int g = g0; g < g1; ++g) local += units_of(g);
@@ -294,7 +296,9 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         uint32_t phase = 0, armed = 0, armed_par = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
-            const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
+            Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
+            const int kb0 = (w.mb / MB) * KB;   // first k-block of this unit's K range
+            w.mb %= MB;
             const int a_row = DUAL ? (w.g * MB + w.mb) * 256 : w.g * p.n_out + w.mb * 128;
             const int b_row = (w.g < E ? offs[w.g] : p.shared_in_row) + w.nb * w.nt;
             const int ti = tile_index(w.nt);
@@ -321,10 +325,11 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 if (!ok) break;
                 const uint32_t fb = smem_u32(&full[stage]);
                 uint8_t* a_s = tiles + (size_t)stage * STAGE_B;
-                const int b_k = p.k_wrap ? (kb % p.k_wrap) : kb;
+                const int kg = kb0 + kb;   // k-block within the whole K
+                const int b_k = p.k_wrap ? (kg % p.k_wrap) : kg;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(fb, tx);
-                    tma_load_2d(smem_u32(a_s), &maps.w, kb * BK, a_row, fb, pol_w);
+                    tma_load_2d(smem_u32(a_s), &maps.w, kg * BK, a_row, fb, pol_w);
                     if (!gather) tma_load_2d(smem_u32(a_s + C::A_BYTES), bm, b_k * BK, b_row, fb, pol_a);
                 }
                 __syncwarp(pmask);
@@ -395,7 +400,9 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
-            const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
+            Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
+            const int kp = w.mb / MB;   // K range of this unit (partial output kp)
+            w.mb %= MB;
             const int rows = group_rows(w.g, E, p.T, offs);
             const int out_base = (w.g < E ? offs[w.g] : p.shared_out_row) + w.nb * w.nt;
             const int nvalid = min(w.nt, rows - w.nb * w.nt);
@@ -411,7 +418,8 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                     tmem_ld_x16_wait(t_row + c0, g16);
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        if (c0 + j < nvalid && keep) p.out_f32[dst0 + (size_t)(c0 + j) * p.out_ld] = __uint_as_float(g16[j]);
+                        if (c0 + j < nvalid && keep)
+                            p.out_f32[kp * p.split_stride + dst0 + (size_t)(c0 + j) * p.out_ld] = __uint_as_float(g16[j]);
                 }
                 tc_fence_before();
                 mbar_arrive(smem_u32(&tempty[acc]));
@@ -848,19 +856,20 @@ cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const u
     for (int i = 0; i < kNumTiles; ++i) m2.sh[i] = m2.act[i];
 
     GemmParams p1{offsets, E, (int)T, (int)routed, H, I, 0, (int)routed, nt, 0, 0, I, I, gather ? row_token : nullptr,
-                  h, nullptr, err};
+                  1, 0, h, nullptr, err};
     cudaError_t e = pairs ? run_gemm_pair<MODE_GATEUP>(m1, p1, num_sms, s) : run_gemm<MODE_GATEUP>(m1, p1, num_sms, s);
     if (e != cudaSuccess) return e;
-    GemmParams p2{offsets, E, (int)T, (int)routed, I, H, (int)routed, (int)routed, nt, 0, 0, H, H, nullptr, y, nullptr,
-                  err};
+    GemmParams p2{offsets, E, (int)T, (int)routed, I, H, (int)routed, (int)routed, nt, 0, 0, H, H, nullptr, 1, 0, y,
+                  nullptr, err};
     e = pairs ? run_gemm_pair<MODE_DOWN>(m2, p2, num_sms, s) : run_gemm<MODE_DOWN>(m2, p2, num_sms, s);
     if (e == cudaSuccess) launches_add(2);
     return e;
 }
 
-// Router logits on the tensor cores: logits[T][E] = x [T][H] . (W_hi + W_mid + W_lo)^T, where
-// w_split [e_pad][3H] holds the three bf16 pieces of each fp32 router row side by side (rows
-// >= E are zero). One group of T rows; the K loop runs over 3H while x's K coordinate wraps.
+// Router logits on the tensor cores: partial[p][T][E] = x [T][H] . W_p^T for the three bf16
+// pieces p = hi, mid, lo of W_r; w_split [e_pad][3H] holds the pieces of each fp32 router row
+// side by side (rows >= E are zero). One group of T rows; each unit covers one piece's K range
+// (x's K coordinate wraps), so the three partials are summed later in a fixed order.
 cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* w_split, int e_pad, int E,
                                float* logits, int nt, int num_sms, cudaStream_t s) {
     constexpr int BK = SMOE_GEMM_BK;
@@ -869,7 +878,8 @@ cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16
         !make_act_maps(m.sh, x, (uint64_t)T, H, nt, BK))
         return cudaErrorNotSupported;
     for (int i = 0; i < kNumTiles; ++i) m.act[i] = m.sh[i];
-    GemmParams p{nullptr, 0, (int)T, 0, 3 * H, e_pad, 0, 0, nt, 0, H / BK, E, E, nullptr, nullptr, logits, nullptr};
+    GemmParams p{nullptr, 0, (int)T, 0, 3 * H, e_pad, 0, 0, nt, 0, H / BK, E, E, nullptr, 3, (size_t)T * E, nullptr,
+                 logits, nullptr};
     return run_gemm<MODE_ROUTER>(m, p, num_sms, s);
 }
 

@@ -236,7 +236,15 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
         }
         const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
         uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * H);
-        for (int c = lane; c < vec; c += 32) dst[c] = src[c];
+        int c = lane;
+        for (; c + 96 < vec; c += 128) {   // four 16-byte vectors in flight per lane
+            const uint4 a = src[c], b = src[c + 32], d = src[c + 64], e = src[c + 96];
+            dst[c] = a;
+            dst[c + 32] = b;
+            dst[c + 64] = d;
+            dst[c + 96] = e;
+        }
+        for (; c < vec; c += 32) dst[c] = src[c];
     }
 }
 

@@ -315,9 +315,9 @@ RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms, bool allo
         p.e_pad = (E + 127) / 128 * 128;
         const int mb = p.e_pad / 128;
         p.nt = 256;
-        while (p.nt > 64 && ((T + p.nt - 1) / p.nt) * mb < num_sms) p.nt /= 2;
-        p.splits = 1;
-        const size_t logit_b = ((size_t)T * E * 4 + 255) / 256 * 256;
+        while (p.nt > 64 && ((T + p.nt - 1) / p.nt) * mb * 3 < num_sms) p.nt /= 2;
+        p.splits = 3;   // one partial per bf16 piece of W_r, summed in order by the top-k kernel
+        const size_t logit_b = ((size_t)3 * T * E * 4 + 255) / 256 * 256;
         p.scratch_bytes = logit_b + (size_t)p.e_pad * 3 * c.hidden * 2;
         return p;
     }
@@ -348,7 +348,7 @@ cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, c
     cudaError_t e;
     int n = 2;
     if (p.tc) {
-        const size_t logit_b = ((size_t)T * E * 4 + 255) / 256 * 256;
+        const size_t logit_b = ((size_t)3 * T * E * 4 + 255) / 256 * 256;
         uint16_t* w_split = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(partials) + logit_b);
         {
             LaunchTimer lt(K_ROUTER_SPLIT, s);
