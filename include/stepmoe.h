@@ -28,7 +28,7 @@
  *     no host<->device synchronisation inside any call except smoe_get_device_error.
  *   - No exceptions cross the ABI. T == 0 is a no-op returning SMOE_OK.
  *   - Supported shapes: hidden, inter multiples of 128; shared_inter == inter;
- *     1 <= top_k <= min(32, n_experts); n_experts <= 1024; swiglu_limit == 0.
+ *     1 <= top_k <= min(32, n_experts); n_experts <= 1024.
  *     Anything else returns SMOE_ERR_UNSUPPORTED before any work is enqueued.
  *   - Bad data found on the device (an expert index out of range, a duplicate expert in a
  *     token's selection, a row index out of range) is skipped, never dereferenced, and
@@ -71,8 +71,14 @@ typedef struct {
     int32_t inter;         /* I: routed expert intermediate width (1280)    */
     int32_t shared_inter;  /* Is: shared expert intermediate width (1280)   */
     float route_scale;     /* factor applied to the normalised weights (3)  */
-    float swiglu_limit;    /* activation clamp; 0 = off (only 0 supported)  */
+    float swiglu_limit;    /* SwiGLU clamp of the routed experts; 0 = off   */
+    float swiglu_limit_shared; /* SwiGLU clamp of the shared expert; 0 = off */
 } smoe_config_t;
+/* SwiGLU clamp (model card raw config fields swiglu_limits, swiglu_limits_shared: 0 for most
+ * layers, 7 (routed) and 16 (shared) for the deepest ones; activation clipping against
+ * localized activation blow-up, paperlayer.ai summary §4.1.3 and §B). The pages do not spell out
+ * the clamp; read here as: with limit L > 0, gate g = min(g, L) and up u = clamp(u, -L, L) before
+ * h = SiLU(g) * u. Limits must be finite and >= 0. */
 
 /* Human-readable name of a status code. Never NULL. */
 SMOE_API const char* smoe_status_string(smoe_status_t status);

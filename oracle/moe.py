@@ -32,7 +32,11 @@ Readings where the pages are silent (each is also listed in the design notes):
    smaller expert index first;
 6. a token is a near tie when its 8th and 9th biased scores differ by less than 1e-5; any
    selection within that band is correct there (``valid_selections``);
-7. the layer output is the FFN output only (no residual, no norm).
+7. the layer output is the FFN output only (no residual, no norm);
+8. SwiGLU clamp (model card fields ``swiglu_limits`` / ``swiglu_limits_shared``, garbled on the
+   page; paperlayer.ai §4.1.3 and §B name activation clipping): with limit L > 0 the gate is
+   clamped from above, min(g, L), and the up projection on both sides, clamp(u, -L, L), before
+   SiLU(g) * u. L = 0 means no clamp. Routed and shared experts have their own limits.
 
 Everything is computed in fp64 with no intermediate rounding. bf16 inputs and fp32 router
 weights are exact in fp64.
@@ -175,30 +179,38 @@ def silu(z: np.ndarray) -> np.ndarray:
     return z / (1.0 + np.exp(-z))
 
 
-def swiglu_ffn(X: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray) -> np.ndarray:
-    """F(x) = W_d (SiLU(W_g x) * (W_u x)) for each row x of X (all fp64)."""
-    h = silu(X @ Wg.T) * (X @ Wu.T)
-    return h @ Wd.T
+def swiglu_hidden(X: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, limit: float = 0.0) -> np.ndarray:
+    """The SwiGLU hidden activation SiLU(W_g x) * (W_u x) for each row x of X; with limit L > 0
+    the gate is clamped to (-inf, L] and the up projection to [-L, L] first (reading 8)."""
+    G = X @ Wg.T
+    U = X @ Wu.T
+    if limit > 0.0:
+        G = np.minimum(G, limit)
+        U = np.clip(U, -limit, limit)
+    return silu(G) * U
 
 
-def swiglu_hidden(X: np.ndarray, Wg: np.ndarray, Wu: np.ndarray) -> np.ndarray:
-    """The SwiGLU hidden activation SiLU(W_g x) * (W_u x) for each row x of X."""
-    return silu(X @ Wg.T) * (X @ Wu.T)
+def swiglu_ffn(X: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray, limit: float = 0.0) -> np.ndarray:
+    """F(x) = W_d (SiLU(W_g x) * (W_u x)) for each row x of X (all fp64), clamped as in
+    swiglu_hidden when limit > 0."""
+    return swiglu_hidden(X, Wg, Wu, limit) @ Wd.T
 
 
 ExpertFn = Callable[[int], Sequence[np.ndarray]]   # e -> (W_g, W_u, W_d) fp64; e == E is shared
 
 
-def moe_sparse(x: np.ndarray, r: Route, expert: ExpertFn, E: int) -> np.ndarray:
+def moe_sparse(x: np.ndarray, r: Route, expert: ExpertFn, E: int, limit: float = 0.0,
+               limit_shared: float = 0.0) -> np.ndarray:
     """out[t] = F_shared(x_t) + sum_j w[t, j] F_{idx[t, j]}(x_t), computing only selected experts."""
-    out = swiglu_ffn(x, *expert(E))
+    out = swiglu_ffn(x, *expert(E), limit=limit_shared)
     for e in np.unique(r.idx):
         rows, slots = np.nonzero(r.idx == e)
-        out[rows] += r.w[rows, slots][:, None] * swiglu_ffn(x[rows], *expert(int(e)))
+        out[rows] += r.w[rows, slots][:, None] * swiglu_ffn(x[rows], *expert(int(e)), limit=limit)
     return out
 
 
-def moe_dense_masked(x: np.ndarray, r: Route, expert: ExpertFn, E: int) -> np.ndarray:
+def moe_dense_masked(x: np.ndarray, r: Route, expert: ExpertFn, E: int, limit: float = 0.0,
+                     limit_shared: float = 0.0) -> np.ndarray:
     """out[t] = F_shared(x_t) + sum_e m[t, e] w[t, e] F_e(x_t) over all E experts (0/1 mask m)."""
     T, k = r.idx.shape
     m = np.zeros((T, E))
@@ -206,20 +218,20 @@ def moe_dense_masked(x: np.ndarray, r: Route, expert: ExpertFn, E: int) -> np.nd
     for j in range(k):
         m[np.arange(T), r.idx[:, j]] = 1.0
         wfull[np.arange(T), r.idx[:, j]] = r.w[:, j]
-    out = swiglu_ffn(x, *expert(E))
+    out = swiglu_ffn(x, *expert(E), limit=limit_shared)
     for e in range(E):
-        out += (m[:, e] * wfull[:, e])[:, None] * swiglu_ffn(x, *expert(e))
+        out += (m[:, e] * wfull[:, e])[:, None] * swiglu_ffn(x, *expert(e), limit=limit)
     return out
 
 
 def moe_given_selection(x_t: np.ndarray, s_t: np.ndarray, sel: Sequence[int], expert: ExpertFn, E: int,
-                        scale: float) -> np.ndarray:
+                        scale: float, limit: float = 0.0, limit_shared: float = 0.0) -> np.ndarray:
     """Output row of one token for a given selected set (used for near-tie tokens)."""
     sel = list(sel)
     w = normalise(s_t[sel], scale)
-    out = swiglu_ffn(x_t[None, :], *expert(E))[0]
+    out = swiglu_ffn(x_t[None, :], *expert(E), limit=limit_shared)[0]
     for wj, e in zip(w, sel):
-        out = out + wj * swiglu_ffn(x_t[None, :], *expert(e))[0]
+        out = out + wj * swiglu_ffn(x_t[None, :], *expert(e), limit=limit)[0]
     return out
 
 

@@ -25,7 +25,7 @@ SMOE_ERR_CUDA, SMOE_ERR_DEVICE, SMOE_ERR_TIMEOUT = 4, 5, 6
 class SmoeConfig(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int32), ("n_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("inter", ctypes.c_int32), ("shared_inter", ctypes.c_int32), ("route_scale", ctypes.c_float),
-                ("swiglu_limit", ctypes.c_float)]
+                ("swiglu_limit", ctypes.c_float), ("swiglu_limit_shared", ctypes.c_float)]
 
 
 class SmoeError(RuntimeError):
@@ -35,8 +35,8 @@ class SmoeError(RuntimeError):
 
 
 def config(hidden=4096, n_experts=288, top_k=8, inter=1280, shared_inter=1280, route_scale=3.0,
-           swiglu_limit=0.0) -> SmoeConfig:
-    return SmoeConfig(hidden, n_experts, top_k, inter, shared_inter, route_scale, swiglu_limit)
+           swiglu_limit=0.0, swiglu_limit_shared=0.0) -> SmoeConfig:
+    return SmoeConfig(hidden, n_experts, top_k, inter, shared_inter, route_scale, swiglu_limit, swiglu_limit_shared)
 
 
 class SmoeKernelTime(ctypes.Structure):

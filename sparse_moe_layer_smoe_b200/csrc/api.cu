@@ -159,11 +159,13 @@ smoe_status_t smoe_check_config(const smoe_config_t* c) {
     if (c == nullptr) return SMOE_ERR_INVALID_ARG;
     if (c->hidden <= 0 || c->n_experts <= 0 || c->top_k <= 0 || c->inter <= 0 || c->shared_inter <= 0)
         return SMOE_ERR_INVALID_ARG;
-    if (!(c->route_scale > 0.0f) || !isfinite(c->route_scale) || isnan(c->swiglu_limit)) return SMOE_ERR_INVALID_ARG;
+    if (!(c->route_scale > 0.0f) || !isfinite(c->route_scale)) return SMOE_ERR_INVALID_ARG;
+    if (!(c->swiglu_limit >= 0.0f) || !isfinite(c->swiglu_limit) || !(c->swiglu_limit_shared >= 0.0f) ||
+        !isfinite(c->swiglu_limit_shared))
+        return SMOE_ERR_INVALID_ARG;
     if (c->hidden % 128 != 0 || c->inter % 128 != 0 || c->shared_inter != c->inter) return SMOE_ERR_UNSUPPORTED;
     if (c->n_experts > 1024 || c->top_k > 32 || c->top_k > c->n_experts) return SMOE_ERR_UNSUPPORTED;
     if (c->hidden > 32768 || c->inter > 32768) return SMOE_ERR_UNSUPPORTED;
-    if (c->swiglu_limit != 0.0f) return SMOE_ERR_UNSUPPORTED;
     return SMOE_OK;
 }
 

@@ -77,6 +77,8 @@ struct GemmParams {
     int out_ld;               // leading dimension of the output rows
     int out_valid;            // output features stored: f < out_valid
     const int32_t* row_token; // gather mode (routed groups read x rows by token), else nullptr
+    float clamp_routed;       // SwiGLU clamp limit of routed groups (0 = off)
+    float clamp_shared;       // SwiGLU clamp limit of the shared group (0 = off)
     int ksplit;               // K split into this many equal ranges, one unit each (router pieces)
     size_t split_stride;      // elements between the partial outputs of consecutive K ranges
     uint16_t* out;            // [*, out_ld] bf16 (gate/up, down)
@@ -143,10 +145,11 @@ __device__ __forceinline__ Unit decode_unit(int u, const int32_t* prefix, const 
 }
 
 // Epilogue, part 1: drain this thread's accumulator row (one output feature, up to 256 token
-// columns) into registers as packed bf16 pairs: SiLU(gate) * up for gate/up, the plain value for
-// down. 32-column TMEM loads, one wait each. nch = number of 32-column chunks holding valid tokens.
+// columns) into registers as packed bf16 pairs: SiLU(gate) * up for gate/up (after the SwiGLU
+// clamp when lim > 0), the plain value for down. 32-column TMEM loads, one wait each.
+// nch = number of 32-column chunks holding valid tokens.
 template <bool DUAL>
-__device__ __forceinline__ void epi_load(uint32_t t_row, int nt_max, int nch, uint32_t (&hv)[128]) {
+__device__ __forceinline__ void epi_load(uint32_t t_row, int nt_max, int nch, float lim, uint32_t (&hv)[128]) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         if (c < nch) {
@@ -159,8 +162,15 @@ __device__ __forceinline__ void epi_load(uint32_t t_row, int nt_max, int nch, ui
             for (int j = 0; j < 16; ++j) {
                 float v0 = __uint_as_float(a[2 * j]), v1 = __uint_as_float(a[2 * j + 1]);
                 if (DUAL) {
-                    v0 = silu_mul(v0, __uint_as_float(b[2 * j]));
-                    v1 = silu_mul(v1, __uint_as_float(b[2 * j + 1]));
+                    float u0 = __uint_as_float(b[2 * j]), u1 = __uint_as_float(b[2 * j + 1]);
+                    if (lim > 0.0f) {   // SwiGLU clamp: gate from above, up on both sides
+                        v0 = fminf(v0, lim);
+                        v1 = fminf(v1, lim);
+                        u0 = fminf(fmaxf(u0, -lim), lim);
+                        u1 = fminf(fmaxf(u1, -lim), lim);
+                    }
+                    v0 = silu_mul(v0, u0);
+                    v1 = silu_mul(v1, u1);
                 }
                 hv[16 * c + j] = (uint32_t)float_to_bf16_bits(v0) | ((uint32_t)float_to_bf16_bits(v1) << 16);
             }
@@ -426,7 +436,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             } else {
                 const int nch = (nvalid + 31) / 32;
                 uint32_t hv[128];
-                epi_load<DUAL>(t_row, p.nt_max, nch, hv);
+                epi_load<DUAL>(t_row, p.nt_max, nch, w.g < E ? p.clamp_routed : p.clamp_shared, hv);
                 tc_fence_before();
                 mbar_arrive(smem_u32(&tempty[acc]));   // accumulator free before the stores
                 epi_store(hv, nch, nvalid, p.out, dst0, p.out_ld);
@@ -659,7 +669,7 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
             const size_t dst0 = (size_t)out_base * p.out_ld + f;
             const int nch = (nvalid + 31) / 32;
             uint32_t hv[128];
-            epi_load<DUAL>(t_row, p.nt_max, nch, hv);
+            epi_load<DUAL>(t_row, p.nt_max, nch, w.g < E ? p.clamp_routed : p.clamp_shared, hv);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));   // accumulator free
@@ -856,11 +866,11 @@ cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const u
     for (int i = 0; i < kNumTiles; ++i) m2.sh[i] = m2.act[i];
 
     GemmParams p1{offsets, E, (int)T, (int)routed, H, I, 0, (int)routed, nt, 0, 0, I, I, gather ? row_token : nullptr,
-                  1, 0, h, nullptr, err};
+                  c.swiglu_limit, c.swiglu_limit_shared, 1, 0, h, nullptr, err};
     cudaError_t e = pairs ? run_gemm_pair<MODE_GATEUP>(m1, p1, num_sms, s) : run_gemm<MODE_GATEUP>(m1, p1, num_sms, s);
     if (e != cudaSuccess) return e;
-    GemmParams p2{offsets, E, (int)T, (int)routed, I, H, (int)routed, (int)routed, nt, 0, 0, H, H, nullptr, 1, 0, y,
-                  nullptr, err};
+    GemmParams p2{offsets, E, (int)T, (int)routed, I, H, (int)routed, (int)routed, nt, 0, 0, H, H, nullptr, 0.f, 0.f, 1,
+                  0, y, nullptr, err};
     e = pairs ? run_gemm_pair<MODE_DOWN>(m2, p2, num_sms, s) : run_gemm<MODE_DOWN>(m2, p2, num_sms, s);
     if (e == cudaSuccess) launches_add(2);
     return e;
@@ -878,8 +888,8 @@ cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16
         !make_act_maps(m.sh, x, (uint64_t)T, H, nt, BK))
         return cudaErrorNotSupported;
     for (int i = 0; i < kNumTiles; ++i) m.act[i] = m.sh[i];
-    GemmParams p{nullptr, 0, (int)T, 0, 3 * H, e_pad, 0, 0, nt, 0, H / BK, E, E, nullptr, 3, (size_t)T * E, nullptr,
-                 logits, nullptr};
+    GemmParams p{nullptr, 0, (int)T, 0, 3 * H, e_pad, 0, 0, nt, 0, H / BK, E, E, nullptr, 0.f, 0.f, 3, (size_t)T * E,
+                 nullptr, logits, nullptr};
     return run_gemm<MODE_ROUTER>(m, p, num_sms, s);
 }
 

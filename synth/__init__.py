@@ -17,6 +17,7 @@ Workloads (Step 3.5 Flash model card, raw config fields ``hidden_size 4096``,
 * ``prefill``  T=8192, Step shape, bias 0
 * ``skewed``   T=4096, Step shape, Zipf(1.2) popularity bias, 16 dead experts
 * ``mtp``      T=512 (128 sequences x 4 tokens), 1% of rows (5) scaled x50
+* ``mtp_clamp`` the MTP batch with the SwiGLU clamp of the deepest layers (routed 7, shared 16)
 
 x ~ N(0, 1) -> bf16; router W_r ~ N(0, 0.02) fp32; expert weights ~ N(0, 0.02) -> bf16.
 """
@@ -209,6 +210,8 @@ class Workload:
     bias: str = "zero"            # "zero" | "zipf"
     spike_rows: int = 0           # rows of x scaled x spike_mult
     spike_mult: float = 50.0
+    swiglu_limit: float = 0.0           # SwiGLU clamp of routed experts (0 = off)
+    swiglu_limit_shared: float = 0.0    # SwiGLU clamp of the shared expert (0 = off)
     seed: int = 0
     x_std: float = 1.0
     w_std: float = 0.02
@@ -226,6 +229,11 @@ WORKLOADS = {
                        description="T=4096, Zipf(1.2) expert popularity via router bias, 16 dead experts"),
     "mtp": Workload("mtp", 512, 4096, 288, 8, 1280, 1280, spike_rows=5,
                     description="MTP-3 verify batch 128x4=512 tokens, 1% of rows x50"),
+    # the clamped variant of the deepest layers (model card swiglu_limits 7, swiglu_limits_shared
+    # 16) on the MTP batch, whose x50 spike rows drive activations past the limits
+    "mtp_clamp": Workload("mtp_clamp", 512, 4096, 288, 8, 1280, 1280, spike_rows=5, swiglu_limit=7.0,
+                          swiglu_limit_shared=16.0,
+                          description="MTP verify batch with the SwiGLU clamp (routed 7, shared 16)"),
     # profiling case: the decode kernel shape (~2 rows per expert) on 32 experts, ~1 GB of weights
     "decode_e32": Workload("decode_e32", 8, 4096, 32, 8, 1280, 1280,
                            description="decode-shaped small case for counter captures: T=8, 32 experts top-8"),

@@ -23,7 +23,12 @@ ALL_WORKLOADS = ["tiny"] + STEP_WORKLOADS
 
 def cfg_of(w: synth.Workload):
     import sparse_moe_layer_smoe_b200 as smoe
-    return smoe.config(w.H, w.E, w.k, w.I, w.Is, w.route_scale, 0.0)
+    return smoe.config(w.H, w.E, w.k, w.I, w.Is, w.route_scale, w.swiglu_limit, w.swiglu_limit_shared)
+
+
+def limit_of(w: synth.Workload, g: int) -> float:
+    """SwiGLU clamp limit of group g (g == E: the shared expert)."""
+    return w.swiglu_limit_shared if g == w.E else w.swiglu_limit
 
 
 def shape_key(w: synth.Workload):

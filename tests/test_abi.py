@@ -32,7 +32,10 @@ def test_status_strings():
     ("hidden", -128, smoe.SMOE_ERR_INVALID_ARG),
     ("route_scale", 0.0, smoe.SMOE_ERR_INVALID_ARG),
     ("route_scale", float("inf"), smoe.SMOE_ERR_INVALID_ARG),
-    ("swiglu_limit", 7.0, smoe.SMOE_ERR_UNSUPPORTED),
+    ("swiglu_limit", -1.0, smoe.SMOE_ERR_INVALID_ARG),
+    ("swiglu_limit", float("nan"), smoe.SMOE_ERR_INVALID_ARG),
+    ("swiglu_limit_shared", float("inf"), smoe.SMOE_ERR_INVALID_ARG),
+    ("swiglu_limit", 7.0, smoe.SMOE_OK),
 ])
 def test_config_validation(field, value, expect):
     c = smoe.config()

@@ -18,7 +18,7 @@ import pytest
 import oracle
 import synth
 from layer_fixtures import (ALL_WORKLOADS, HostExperts, assert_close, bf16_tensor_to_f64, cfg_of, device_inputs,
-                            host_route, host_x64, selection_ok)
+                            host_route, host_x64, limit_of, selection_ok)
 
 pytestmark = pytest.mark.gpu
 
@@ -131,7 +131,7 @@ def _ffn_sample_rows(offsets, T, k, n_groups=6):
 
 
 @pytest.mark.parametrize("mode", ["gather", "x_perm"])
-@pytest.mark.parametrize("name", ALL_WORKLOADS)
+@pytest.mark.parametrize("name", ALL_WORKLOADS + ["mtp_clamp"])
 def test_expert_ffn_parity(name, mode):
     """gather: routed rows read from x through row_token inside the GEMM; x_perm: from a
     permuted copy of x built on the host from the oracle's permutation."""
@@ -154,14 +154,24 @@ def test_expert_ffn_parity(name, mode):
     experts = HostExperts(w)
     group_of = np.searchsorted(offsets, np.arange(T * k), side="right") - 1
     rows = list(range(T * k + T)) if name == "tiny" else _ffn_sample_rows(offsets, T, k)
+    spikes = synth.spike_rows(w)
+    if len(spikes):   # rows of the x50 spike tokens: routed ones and their shared rows
+        rows = sorted(set(rows) | set(np.nonzero(np.isin(row_token, spikes))[0][:6].tolist())
+                      | set((T * k + spikes[:2]).tolist()))
     ref = np.empty((len(rows), w.H))
     by_group = {}
     for i, rr in enumerate(rows):
         g, tok = (E, rr - T * k) if rr >= T * k else (int(group_of[rr]), int(row_token[rr]))
         by_group.setdefault(g, []).append((i, tok))
+    clamped = 0.0
     for g, items in by_group.items():
         ii = [a for a, _ in items]
-        ref[ii] = oracle.swiglu_ffn(x64[[b for _, b in items]], *experts(g))
+        xs = x64[[b for _, b in items]]
+        ref[ii] = oracle.swiglu_ffn(xs, *experts(g), limit=limit_of(w, g))
+        if limit_of(w, g) > 0:
+            clamped = max(clamped, np.abs(ref[ii] - oracle.swiglu_ffn(xs, *experts(g))).max())
+    if w.swiglu_limit > 0:
+        assert clamped > 0.0   # the sampled rows exercise the clamp
     assert np.all(np.isfinite(gy[rows]))
     fro, mx = assert_close(gy[rows], ref, f"{name} expert_ffn ({mode})")
     assert torch.isfinite(y.float()).all()   # every row written
@@ -212,15 +222,16 @@ def _layer_rows(name, rows, gi, w, dense):
         assert ok, f"token {t}: selection {gset}"
         sel_rows.append((t, ref_set))
     sub = oracle.Route(r.logits[rows], r.s[rows], r.bhat[rows], r.idx[rows], r.w[rows], r.gap[rows])
+    lim = dict(limit=w.swiglu_limit, limit_shared=w.swiglu_limit_shared)
     if dense:
-        ref = oracle.moe_dense_masked(x64[rows], sub, experts, w.E)
+        ref = oracle.moe_dense_masked(x64[rows], sub, experts, w.E, **lim)
     else:
-        ref = oracle.moe_sparse(x64[rows], sub, experts, w.E)
+        ref = oracle.moe_sparse(x64[rows], sub, experts, w.E, **lim)
     for i, (t, ref_set) in enumerate(sel_rows):
         if ref_set != tuple(sorted(r.idx[t].tolist())):
             # near tie resolved to another valid set: the oracle's output for that set
             order = sorted(ref_set, key=lambda e: -r.bhat[t, e])
-            ref[i] = oracle.moe_given_selection(x64[t], r.s[t], order, experts, w.E, w.route_scale)
+            ref[i] = oracle.moe_given_selection(x64[t], r.s[t], order, experts, w.E, w.route_scale, **lim)
     return ref
 
 
@@ -239,7 +250,7 @@ def test_forward_parity_dense_masked(name):
     print(f"{name}: forward rel_fro={fro:.2e} rel_max={mx:.2e}")
 
 
-@pytest.mark.parametrize("name", ["prefill", "skewed", "mtp"])
+@pytest.mark.parametrize("name", ["prefill", "skewed", "mtp", "mtp_clamp"])
 def test_forward_parity_sampled(name):
     w, out, _ = _forward(name)
     cfg = cfg_of(w)

@@ -289,6 +289,50 @@ def test_three_matrix_expert_shape_from_parameter_budget():
     assert 3 * H * I * 9 * layers < 11e9
 
 
+@pytest.mark.parametrize("L", [0.5, 2.0, 7.0])
+def test_swiglu_clamp_brute_force_loops(L):
+    H, I = 6, 4
+    x = 4.0 * RNG.standard_normal((3, H))   # large enough that gate and up cross +-L
+    Wg, Wu, Wd = RNG.standard_normal((I, H)), RNG.standard_normal((I, H)), RNG.standard_normal((H, I))
+    Y = oracle.swiglu_ffn(x, Wg, Wu, Wd, limit=L)
+    crossed = 0
+    for t in range(3):
+        h = []
+        for i in range(I):
+            g = sum(Wg[i, c] * x[t, c] for c in range(H))
+            u = sum(Wu[i, c] * x[t, c] for c in range(H))
+            crossed += (g > L) + (abs(u) > L) + (g < -L)
+            g = g if g < L else L
+            u = -L if u < -L else (L if u > L else u)
+            h.append(g / (1.0 + math.exp(-g)) * u)
+        for o in range(H):
+            assert abs(Y[t, o] - sum(Wd[o, i] * h[i] for i in range(I))) < 1e-11
+    assert crossed > 0
+
+
+def test_swiglu_clamp_closed_forms_and_limits():
+    eye = np.eye(2)
+    # gate 10 clamped to 3, up 10 clamped to 3: SiLU(3) * 3 on the diagonal
+    Y = oracle.swiglu_ffn(np.array([[10.0, -10.0]]), eye, eye, eye, limit=3.0)
+    s3 = 3.0 / (1.0 + math.exp(-3.0))
+    assert abs(Y[0, 0] - s3 * 3.0) < 1e-15
+    # gate -10 is not clamped from below: SiLU(-10) * (-3)
+    assert abs(Y[0, 1] - (-10.0 / (1.0 + math.exp(10.0))) * -3.0) < 1e-15
+    # no clamp for L = 0 and for a limit above every activation
+    x, wr, experts = _tiny_layer()
+    for e in range(3):
+        a = oracle.swiglu_ffn(x, *experts[e])
+        assert np.array_equal(oracle.swiglu_ffn(x, *experts[e], limit=0.0), a)
+        assert np.array_equal(oracle.swiglu_ffn(x, *experts[e], limit=1e9), a)
+    # the layer applies the routed limit to routed experts and the shared limit to the shared one
+    r = oracle.route(x, wr, np.zeros(6), 2, 3.0)
+    big = oracle.moe_sparse(x, r, lambda e: experts[e], 6, limit=1e9, limit_shared=1e9)
+    assert np.array_equal(big, oracle.moe_sparse(x, r, lambda e: experts[e], 6))
+    only_shared = oracle.moe_sparse(x, r, lambda e: experts[e], 6, limit=1e9, limit_shared=0.01)
+    assert np.allclose(only_shared - big, oracle.swiglu_ffn(x, *experts[6], limit=0.01) - oracle.swiglu_ffn(
+        x, *experts[6]), rtol=1e-12, atol=1e-13)
+
+
 # ------------------------------------------------------------------ planted mistakes
 def _pins_fail(monkeypatch, name, fn, test, *args):
     monkeypatch.setattr(oracle, name, fn)
@@ -322,3 +366,14 @@ def test_pins_catch_wrong_silu_sign(monkeypatch):
     monkeypatch.setattr(oracle, "silu", lambda z: z / (1.0 + np.exp(z)))
     with pytest.raises(AssertionError):
         test_silu_closed_forms()
+
+
+def test_pins_catch_gate_clamped_from_below(monkeypatch):
+    def bad(X, Wg, Wu, Wd, limit=0.0):
+        G, U = X @ Wg.T, X @ Wu.T
+        if limit > 0:
+            G, U = np.clip(G, -limit, limit), np.clip(U, -limit, limit)
+        return (oracle.moe.silu(G) * U) @ Wd.T
+    monkeypatch.setattr(oracle, "swiglu_ffn", bad)
+    with pytest.raises(AssertionError):
+        test_swiglu_clamp_brute_force_loops(0.5)
