@@ -76,7 +76,10 @@ int choose_token_tile(const smoe_config_t& c, int64_t T);
 
 // smoe_forward reads routed rows straight from x (TMA row gathers) when the largest token tile
 // is at most this; above it, per-row gathers cost more than one gather kernel plus tile loads.
-constexpr int kGatherMaxTile = 32;
+#ifndef SMOE_GATHER_MAX_TILE
+#define SMOE_GATHER_MAX_TILE 32
+#endif
+constexpr int kGatherMaxTile = SMOE_GATHER_MAX_TILE;
 
 // x_perm == nullptr selects gather mode: routed rows are read from x through row_token.
 // Returns cudaErrorNotSupported when the driver entry point for tensor maps is unavailable.

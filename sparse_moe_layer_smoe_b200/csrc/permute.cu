@@ -296,7 +296,7 @@ cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int6
     if (x != nullptr && x_perm != nullptr) {
         const int64_t rows = T * k;
         int64_t blocks = (rows + 7) / 8;
-        if (blocks > 148 * 8) blocks = 148 * 8;
+        if (blocks > 148 * 32) blocks = 148 * 32;
         {
             LaunchTimer lt(K_GATHER_ROWS, s);
             gather_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, row_token, offsets, E, (int)T, c.hidden, x_perm,
