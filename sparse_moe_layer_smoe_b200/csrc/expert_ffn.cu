@@ -55,6 +55,10 @@ constexpr int kMaxStages = SMOE_MAX_STAGES;
 #define SMOE_PAIR_MIN_TILE 64    // CTA pairs for launches whose largest token tile is at least this
 #endif
 constexpr int kPairMinTile = SMOE_PAIR_MIN_TILE;
+#ifndef SMOE_PAIR_PREFETCH
+#define SMOE_PAIR_PREFETCH 0     // CTA pairs: L2 prefetch of the weight tile this many k-blocks ahead (0 = off)
+#endif
+constexpr int kPairPrefetch = SMOE_PAIR_PREFETCH;
 
 struct GemmMaps {
     CUtensorMap w;                  // weights [rows][K]: box {BK, 256 (gate/up) or 128 (down)}
@@ -128,6 +132,11 @@ __device__ __forceinline__ int group_tile(int rows, int nt_max) {
 }
 
 __device__ __forceinline__ int tile_index(int nt) { return 31 - __clz(nt) - 4; }   // 16 -> 0 ... 256 -> 4
+
+// Columns the MMAs of a unit compute: its valid token rows rounded up to 16 (the N step of
+// M=128 and M=256 MMAs), at most the tile. A group of 228 rows loads a 256-row tile but runs
+// N=240 MMAs; the columns past N are never stored.
+__device__ __forceinline__ int mma_cols(int nvalid, int nt) { return min(nt, (nvalid + 15) & ~15); }
 
 __device__ __forceinline__ Unit decode_unit(int u, const int32_t* prefix, const int32_t* offs, int E, int T,
                                             int nt_max) {
@@ -370,7 +379,8 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         bool ok = true;
         for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
             const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
-            const uint32_t idesc = idesc0 | ((uint32_t)(w.nt >> 3) << 17);
+            const int n_mma = mma_cols(group_rows(w.g, E, p.T, offs) - w.nb * w.nt, w.nt);
+            const uint32_t idesc = idesc0 | ((uint32_t)(n_mma >> 3) << 17);
             if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, p.err, abort_flag, true)) break;
             tc_fence_after();
             const uint32_t d = tmem_base + (uint32_t)(acc * ACC_COLS);
@@ -583,11 +593,20 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
         for (int u = pair; ok && u < total; u += npairs) {
             const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);   // w.mb = 256-feature block
             const int a_row = DUAL ? (w.g * MB + 2 * w.mb + (int)rank) * 256 : w.g * p.n_out + w.mb * 256 + (int)rank * 128;
+            // each CTA holds half of the MMA's N columns: the first CTA token rows 0..n/2-1 of the
+            // tile, the second n/2..n-1 (its box of nt/2 rows may run past them; those rows are
+            // never read)
             const int half = w.nt / 2;
-            const int b_row = (w.g < E ? offs[w.g] : p.shared_in_row) + w.nb * w.nt + (int)rank * half;
+            const int n_mma = mma_cols(group_rows(w.g, E, p.T, offs) - w.nb * w.nt, w.nt);
+            const int b_row = (w.g < E ? offs[w.g] : p.shared_in_row) + w.nb * w.nt + (int)rank * (n_mma / 2);
             const int ti = tile_index(w.nt);
             const CUtensorMap* bm = (w.g < E) ? &maps.act[ti] : &maps.sh[ti];
             const uint32_t tx = (uint32_t)(2 * (C::A_BYTES + half * BK * 2));
+            int next_a_row = -1;   // weight rows of this pair's next unit (prefetch target)
+            if (kPairPrefetch > 0 && u + npairs < total) {
+                const Unit nx = decode_unit(u + npairs, prefix, offs, E, p.T, p.nt_max);
+                next_a_row = DUAL ? (nx.g * MB + 2 * nx.mb + (int)rank) * 256 : nx.g * p.n_out + nx.mb * 256 + (int)rank * 128;
+            }
             for (int kb = 0; kb < KB; ++kb) {
                 if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag, true)) { ok = false; break; }
                 const uint32_t fb_local = smem_u32(&full[stage]);
@@ -596,6 +615,13 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
                 uint8_t* a_s = tiles + (size_t)stage * STAGE_B;
                 tma_load_2d_pair(smem_u32(a_s), &maps.w, kb * BK, a_row, fb_leader, pol_w);
                 tma_load_2d_pair(smem_u32(a_s + C::A_BYTES), bm, kb * BK, b_row, fb_leader, pol_a);
+                if (kPairPrefetch > 0) {
+                    const int kp = kb + kPairPrefetch;
+                    if (kp < KB)
+                        tma_prefetch_l2_2d(&maps.w, kp * BK, a_row);
+                    else if (next_a_row >= 0 && kp - KB < KB)
+                        tma_prefetch_l2_2d(&maps.w, (kp - KB) * BK, next_a_row);
+                }
                 armed |= 1u << stage;
                 armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                 if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -615,7 +641,8 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
         bool ok = true;
         for (int u = pair; ok && u < total; u += npairs) {
             const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
-            const uint32_t idesc = idesc0 | ((uint32_t)(w.nt >> 3) << 17);
+            const int n_mma = mma_cols(group_rows(w.g, E, p.T, offs) - w.nb * w.nt, w.nt);
+            const uint32_t idesc = idesc0 | ((uint32_t)(n_mma >> 3) << 17);
             if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, p.err, abort_flag, true)) break;
             tc_fence_after();
             const uint32_t d = tmem_base + (uint32_t)(acc * ACC_COLS);
@@ -881,14 +908,14 @@ cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const u
 // side by side (rows >= E are zero). One group of T rows; each unit covers one piece's K range
 // (x's K coordinate wraps), so the three partials are summed later in a fixed order.
 cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* w_split, int e_pad, int E,
-                               float* logits, int nt, int num_sms, cudaStream_t s) {
+                               float* logits, int nt, int ksplit, int num_sms, cudaStream_t s) {
     constexpr int BK = SMOE_GEMM_BK;
     GemmMaps m;
     if (!make_map(&m.w, w_split, (uint64_t)e_pad, (uint64_t)3 * H, 128, BK) ||
         !make_act_maps(m.sh, x, (uint64_t)T, H, nt, BK))
         return cudaErrorNotSupported;
     for (int i = 0; i < kNumTiles; ++i) m.act[i] = m.sh[i];
-    GemmParams p{nullptr, 0, (int)T, 0, 3 * H, e_pad, 0, 0, nt, 0, H / BK, E, E, nullptr, 0.f, 0.f, 3, (size_t)T * E,
+    GemmParams p{nullptr, 0, (int)T, 0, 3 * H, e_pad, 0, 0, nt, 0, H / BK, E, E, nullptr, 0.f, 0.f, ksplit, (size_t)T * E,
                  nullptr, logits, nullptr};
     return run_gemm<MODE_ROUTER>(m, p, num_sms, s);
 }

@@ -18,6 +18,7 @@ inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a
 // (tc, large T): W_r split into three bf16 pieces in the workspace, token tile nt.
 struct RouterPlan {
     int tm, te, kc, splits;
+    bool wide;              // the 64-token CUDA-core tile
     bool tc;
     int nt, e_pad;
     size_t scratch_bytes;   // partial logits (+ the split weights when tc)
@@ -65,7 +66,7 @@ cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, c
                          int num_sms, cudaStream_t s, bool allow_tc = true);
 
 cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* w_split, int e_pad, int E,
-                               float* logits, int nt, int num_sms, cudaStream_t s);
+                               float* logits, int nt, int ksplit, int num_sms, cudaStream_t s);
 
 cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int64_t T, const uint16_t* x,
                            int32_t* counts, int32_t* offsets, int32_t* perm_row, int32_t* row_token,

@@ -9,13 +9,15 @@
 // Logits, small T (router_logits_kernel): a register-tiled fp32 SGEMM on the CUDA cores. Each
 // CTA owns TM tokens x TE experts over one K range; K is split only when T is small, so the
 // 4.7 MB of W_r is spread over all SMs at decode sizes. Partial sums go to the workspace.
-// Logits, large T (router_split_kernel + the grouped tensor-core GEMM in router mode): W_r is
+// Logits, T >= 512 (router_split_kernel + the grouped tensor-core GEMM in router mode): W_r is
 // split exactly into three bf16 pieces, so x W_r^T = x W_hi^T + x W_mid^T + x W_lo^T with
 // every product exact, accumulated in fp32 in TMEM (19 GFLOP of fp32 at T = 8192 become
-// 58 GFLOP of bf16 on the tensor cores).
+// 58 GFLOP of bf16 on the tensor cores); each piece's K range may be cut into 2 or 4 parts so
+// that small batches still cover the SMs, one partial per part.
 // Kernel 2 (router_topk_kernel): one warp per token adds the K-split partials in a fixed
-// order (deterministic), applies sigmoid and bias, selects top-k by repeated warp argmax
-// with the tie rule (biased score, then larger logit, then smaller index) and normalises.
+// order (deterministic), applies sigmoid and bias, and selects top-k in k rounds of a warp
+// argmax over 64-bit keys (biased score, then logit; warp max reductions), the smaller expert
+// index winning an exact tie; then normalises.
 #include <float.h>
 
 #include "common.cuh"
@@ -149,12 +151,11 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ w
     }
 }
 
-// (b, l, e) is better than (b2, l2, e2): larger biased score, then larger logit, then
-// smaller expert index. NaN scores were mapped to -inf before, so the order is total.
-__device__ __forceinline__ bool better(float b, float l, int e, float b2, float l2, int e2) {
-    if (b != b2) return b > b2;
-    if (l != l2) return l > l2;
-    return e < e2;
+// Order-preserving map of a float to an unsigned key (a < b exactly when key(a) < key(b));
+// -0 is folded into +0 first, as the float comparison treats them as equal.
+__device__ __forceinline__ uint32_t order_key(float f) {
+    const uint32_t u = __float_as_uint(f + 0.0f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 template <int NPL>
@@ -166,76 +167,87 @@ router_topk_kernel(const float* __restrict__ part, int splits, const float* __re
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
 
+    // logits: the K-split partials added in split order 0, 1, 2, ... (the order is fixed, so the
+    // result is deterministic); all loads of a group of G splits are issued before the first add
+    constexpr int G = NPL <= 16 ? 4 : 2;
+    const float* pt = part + (size_t)t * E + lane;
+    const size_t stride = (size_t)T * E;
     float L[NPL], S[NPL], B[NPL];
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
+        L[i] = 0.f;
+        B[i] = (lane + 32 * i < E) ? bias[lane + 32 * i] : 0.f;
+    }
+    for (int s0 = 0; s0 < splits; s0 += G) {
+        float v[G][NPL];
+#pragma unroll
+        for (int q = 0; q < G; ++q)
+#pragma unroll
+            for (int i = 0; i < NPL; ++i)
+                v[q][i] = (s0 + q < splits && lane + 32 * i < E) ? pt[(size_t)(s0 + q) * stride + 32 * i] : 0.f;
+#pragma unroll
+        for (int q = 0; q < G; ++q)
+#pragma unroll
+            for (int i = 0; i < NPL; ++i)
+                if (s0 + q < splits) L[i] += v[q][i];
+    }
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
-        L[i] = -FLT_MAX;
         S[i] = 0.f;
-        B[i] = -INFINITY;
         if (e < E) {
-            // partial sums added in split order 0, 1, 2, ... (four loads in flight at a time)
-            const float* pe = part + (size_t)t * E + e;
-            const size_t stride = (size_t)T * E;
-            float l = 0.f;
-            int s = 0;
-            for (; s + 4 <= splits; s += 4) {
-                const float a = pe[s * stride], b = pe[(s + 1) * stride], c = pe[(s + 2) * stride],
-                            d = pe[(s + 3) * stride];
-                l = (((l + a) + b) + c) + d;
-            }
-            for (; s < splits; ++s) l += pe[s * stride];
-            L[i] = l;
+            const float l = L[i];
             if (logits_out) logits_out[(size_t)t * E + e] = l;
             const float sg = 1.0f / (1.0f + expf(-l));
             S[i] = sg;
-            float bb = sg + bias[e];
+            const float bb = sg + B[i];
             B[i] = (bb != bb) ? -INFINITY : bb;
             if (l != l) L[i] = -FLT_MAX;
         }
     }
 
-    uint32_t taken = 0;
+    // Selection order: larger biased score, then larger logit, then smaller expert index.
+    // Each candidate carries the 64-bit key (key(b^), key(logit)); a taken or absent candidate
+    // has key 0, below every real one (key(-inf) > 0), and k <= E leaves a real one each round.
+    uint32_t kh[NPL], kl[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const bool live = lane + 32 * i < E;
+        kh[i] = live ? order_key(B[i]) : 0u;
+        kl[i] = live ? order_key(L[i]) : 0u;
+    }
     float s_sel = 0.f;   // this lane's copy of the chosen score for slot j == lane
     int e_sel = 0;
     for (int j = 0; j < k; ++j) {
-        float bb = -INFINITY, ll = -FLT_MAX;
-        int ee = 0x7FFFFFFF;
+        // this lane's best: strict comparison in ascending i keeps the smaller index on a tie
+        uint32_t bh = 0, bl = 0;
+        int bi = 0;
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-            const int e = lane + 32 * i;
-            if (e < E && !((taken >> i) & 1u) && better(B[i], L[i], e, bb, ll, ee)) {
-                bb = B[i];
-                ll = L[i];
-                ee = e;
+        for (int i = 0; i < NPL; ++i)
+            if (kh[i] > bh || (kh[i] == bh && kl[i] > bl)) {
+                bh = kh[i];
+                bl = kl[i];
+                bi = i;
             }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float b2 = __shfl_xor_sync(0xFFFFFFFFu, bb, off);
-            const float l2 = __shfl_xor_sync(0xFFFFFFFFu, ll, off);
-            const int e2 = __shfl_xor_sync(0xFFFFFFFFu, ee, off);
-            if (better(b2, l2, e2, bb, ll, ee)) {
-                bb = b2;
-                ll = l2;
-                ee = e2;
-            }
-        }
-        // every lane now holds the winner ee (valid: k <= E, so an untaken expert exists)
+        // warp-wide: the largest key, then the smallest index among the lanes holding it
+        const uint32_t mh = __reduce_max_sync(0xFFFFFFFFu, bh);
+        const uint32_t ml = __reduce_max_sync(0xFFFFFFFFu, bh == mh ? bl : 0u);
+        const uint32_t ee = __reduce_min_sync(0xFFFFFFFFu, (bh == mh && bl == ml) ? (uint32_t)(lane + 32 * bi)
+                                                                                   : 0xFFFFFFFFu);
         float sw = 0.f;
-        if ((ee & 31) == lane) {
-            const int i = ee >> 5;
+        if ((int)(ee & 31u) == lane) {
 #pragma unroll
             for (int q = 0; q < NPL; ++q)
-                if (q == i) {
-                    taken |= 1u << q;
+                if (q == (int)(ee >> 5)) {
+                    kh[q] = 0u;
+                    kl[q] = 0u;
                     sw = S[q];
                 }
         }
-        sw = __shfl_sync(0xFFFFFFFFu, sw, ee & 31);
+        sw = __shfl_sync(0xFFFFFFFFu, sw, ee & 31u);
         if (lane == j) {
             s_sel = sw;
-            e_sel = ee;
+            e_sel = (int)ee;
         }
     }
     // sum of the selected unbiased scores in slot order j = 0..k-1
@@ -251,25 +263,38 @@ router_topk_kernel(const float* __restrict__ part, int splits, const float* __re
 // mid = bf16(w - hi), lo = bf16(w - hi - mid), each difference exact in fp32, so
 // hi + mid + lo reproduces w to about 2^-24 relative and every product with a bf16 x is exact
 // in fp32. Rows e >= E (padding up to a multiple of 128) are zero.
-__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ wr, int E, int e_pad, int H,
+// Grid: (H/4/256 rounded up, e_pad); thread = 4 consecutive elements of row blockIdx.y.
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ wr, int E, int H,
                                                            uint16_t* __restrict__ w_split) {
-    const int64_t n = (int64_t)e_pad * H;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int e = (int)(i / H), h = (int)(i % H);
-        uint16_t p0 = 0, p1 = 0, p2 = 0;
-        if (e < E) {
-            const float w = wr[(size_t)e * H + h];
-            p0 = float_to_bf16_bits(w);
-            const float r1 = w - bf16_bits_to_float(p0);
-            p1 = float_to_bf16_bits(r1);
-            const float r2 = r1 - bf16_bits_to_float(p1);
-            p2 = float_to_bf16_bits(r2);
+    const int e = blockIdx.y;
+    const int c = blockIdx.x * 256 + threadIdx.x;   // 4-element column group
+    if (4 * c >= H) return;
+    float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e < E) w = *reinterpret_cast<const float4*>(wr + (size_t)e * H + 4 * c);
+    const float v[4] = {w.x, w.y, w.z, w.w};
+    uint32_t pc[3][2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        uint32_t h2 = 0, m2 = 0, l2 = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float f = v[2 * q + h];
+            const uint16_t p0 = float_to_bf16_bits(f);
+            const float r1 = f - bf16_bits_to_float(p0);
+            const uint16_t p1 = float_to_bf16_bits(r1);
+            const uint16_t p2 = float_to_bf16_bits(r1 - bf16_bits_to_float(p1));
+            h2 |= (uint32_t)p0 << (16 * h);
+            m2 |= (uint32_t)p1 << (16 * h);
+            l2 |= (uint32_t)p2 << (16 * h);
         }
-        uint16_t* row = w_split + (size_t)e * 3 * H;
-        row[h] = p0;
-        row[H + h] = p1;
-        row[2 * H + h] = p2;
+        pc[0][q] = h2;
+        pc[1][q] = m2;
+        pc[2][q] = l2;
     }
+    uint16_t* row = w_split + (size_t)e * 3 * H + 4 * c;
+#pragma unroll
+    for (int piece = 0; piece < 3; ++piece)
+        *reinterpret_cast<uint2*>(row + (size_t)piece * H) = make_uint2(pc[piece][0], pc[piece][1]);
 }
 
 template <int TM, int TE, int RM, int RE, int KC>
@@ -305,7 +330,15 @@ cudaError_t launch_topk(const float* part, int splits, const float* bias, int64_
 }  // namespace
 
 // Tokens at which the router moves to the tensor cores (3-way bf16 split of W_r).
-constexpr int64_t kRouterTensorCoreMinT = 2048;
+#ifndef SMOE_ROUTER_TC_MIN_T
+#define SMOE_ROUTER_TC_MIN_T 512
+#endif
+constexpr int64_t kRouterTensorCoreMinT = SMOE_ROUTER_TC_MIN_T;
+#ifndef SMOE_ROUTER_WIDE_TILE_MAX_T
+#define SMOE_ROUTER_WIDE_TILE_MAX_T 64
+#endif
+// Batches up to this many tokens use the 64-token router tile.
+constexpr int64_t kRouterWideTileMaxT = SMOE_ROUTER_WIDE_TILE_MAX_T;
 
 RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms, bool allow_tc) {
     RouterPlan p{};
@@ -316,8 +349,12 @@ RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms, bool allo
         const int mb = p.e_pad / 128;
         p.nt = 256;
         while (p.nt > 64 && ((T + p.nt - 1) / p.nt) * mb * 3 < num_sms) p.nt /= 2;
-        p.splits = 3;   // one partial per bf16 piece of W_r, summed in order by the top-k kernel
-        const size_t logit_b = ((size_t)3 * T * E * 4 + 255) / 256 * 256;
+        // K = the three bf16 pieces of W_r, each in m equal ranges: one partial per range,
+        // summed in order by the top-k kernel (m grows until the units cover the SMs)
+        int m = 1;
+        while (m < 4 && c.hidden % (128 * m) == 0 && ((T + p.nt - 1) / p.nt) * mb * 3 * m < num_sms) m *= 2;
+        p.splits = 3 * m;
+        const size_t logit_b = ((size_t)p.splits * T * E * 4 + 255) / 256 * 256;
         p.scratch_bytes = logit_b + (size_t)p.e_pad * 3 * c.hidden * 2;
         return p;
     }
@@ -325,6 +362,13 @@ RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms, bool allo
         p.tm = 64;
         p.te = (E % 96 == 0) ? 96 : 64;
         p.kc = 32;
+    } else if (T <= kRouterWideTileMaxT) {
+        // every token of the batch in one tile: each W_r element is read by one CTA, and each
+        // thread's 4 x 4 register tile takes two 16-byte shared loads per 16 FMAs
+        p.tm = 64;
+        p.te = 32;
+        p.kc = 64;
+        p.wide = true;
     } else {
         p.tm = 16;
         p.te = 32;
@@ -348,15 +392,18 @@ cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, c
     cudaError_t e;
     int n = 2;
     if (p.tc) {
-        const size_t logit_b = ((size_t)3 * T * E * 4 + 255) / 256 * 256;
+        const size_t logit_b = ((size_t)p.splits * T * E * 4 + 255) / 256 * 256;
         uint16_t* w_split = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(partials) + logit_b);
         {
             LaunchTimer lt(K_ROUTER_SPLIT, s);
-            router_split_kernel<<<148 * 4, 256, 0, s>>>(wr, E, p.e_pad, H, w_split);
+            router_split_kernel<<<dim3((unsigned)((H / 4 + 255) / 256), (unsigned)p.e_pad), 256, 0, s>>>(wr, E, H,
+                                                                                                       w_split);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        e = launch_router_gemm(x, T, H, w_split, p.e_pad, E, partials, p.nt, num_sms, s);
+        e = launch_router_gemm(x, T, H, w_split, p.e_pad, E, partials, p.nt, p.splits, num_sms, s);
         n = 3;
+    } else if (p.wide) {
+        e = launch_logits<64, 32, 4, 4, 64>(x, T, wr, E, H, p.splits, partials, s);
     } else if (p.tm == 64 && p.te == 96) {
         e = launch_logits<64, 96, 4, 6, 32>(x, T, wr, E, H, p.splits, partials, s);
     } else if (p.tm == 64) {

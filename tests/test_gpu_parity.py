@@ -90,6 +90,38 @@ def test_route_parity(name):
     print(f"{name}: {near} near-tie tokens of {T}")
 
 
+@pytest.mark.parametrize("T", [37, 700, 2100])   # the small-batch, mid-batch and tensor-core router plans
+def test_route_exact_ties_follow_the_tie_rule(T):
+    """Rows of zeros give every expert the logit 0 and the score 1/2 exactly, so biases drawn
+    from {-1/4, 0, 1/4} tie the biased scores exactly within each bias class: the selection is
+    then fixed by the tie rule alone (larger logit, all equal here, then smaller index) and must
+    match bit for bit, with every weight 3/8. The other rows carry Step-shape inputs."""
+    w = synth.WORKLOADS["decode"]
+    cfg = cfg_of(w)
+    E, k = w.E, w.k
+    wr = device_inputs("decode")[2]
+    xb = synth.host_bf16(T * w.H, 5, synth.TID_X, 1.0).reshape(T, w.H)
+    zero = np.arange(T) % 3 == 0
+    xb[zero] = 0
+    bias = np.random.default_rng(T).choice(np.array([-0.25, 0.0, 0.25], dtype=np.float32), size=E)
+    x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    wt = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    ws = _ws(cfg, T)
+    smoe.smoe_route(cfg, x, T, wr, torch.from_numpy(bias).cuda(), idx, wt, None, ws)
+    gi, gw = idx.cpu().numpy(), wt.cpu().numpy()
+    r = oracle.route(oracle.bf16_to_f64(xb), oracle.f32_to_f64(synth.host_w_router(w)), bias.astype(np.float64), k,
+                     w.route_scale)
+    expect = np.lexsort((np.arange(E), -bias.astype(np.float64)))[:k]
+    for t in np.nonzero(zero)[0]:
+        assert np.array_equal(r.idx[t], expect)
+        assert np.array_equal(gi[t], expect), f"token {t}: {gi[t]} vs {expect}"
+        assert np.all(gw[t] == np.float32(w.route_scale / k))
+    for t in np.nonzero(~zero)[0]:
+        ok, _ = selection_ok(r, t, tuple(sorted(gi[t].tolist())), k)
+        assert ok, f"token {t}"
+
+
 # ------------------------------------------------------------------------------ permute
 @pytest.mark.parametrize("name", ALL_WORKLOADS)
 def test_permute_parity(name):

@@ -10,7 +10,9 @@ run every other test; it also passes when run alone in a fresh process.
 import numpy as np
 import pytest
 
+import oracle
 import synth
+from layer_fixtures import selection_ok
 
 pytestmark = pytest.mark.gpu
 
@@ -42,9 +44,10 @@ def _route_both(w, x, wr, bias):
 def test_route_noalloc_matches_route_on_two_calls_in_a_row():
     w = synth.WORKLOADS["decode"]
     wr, _ = synth.dev_router(w)
-    batches = [("decode", synth.WORKLOADS["decode"]), ("mtp", synth.WORKLOADS["mtp"])]
-    for name, wb in batches:
-        x = synth.dev_x(wb)
+    # both batches below the tensor-core router's size, so both entry points run the same kernels
+    batches = [("decode", synth.WORKLOADS["decode"], 64), ("mtp rows 0-299", synth.WORKLOADS["mtp"], 300)]
+    for name, wb, rows in batches:
+        x = synth.dev_x(wb)[:rows].contiguous()
         bias = torch.from_numpy(synth.host_bias(wb)).cuda()
         r = _route_both(wb, x, wr, bias)
         (i0, w0, l0), (i1, w1, l1) = r["workspace"], r["noalloc"]
@@ -55,6 +58,30 @@ def test_route_noalloc_matches_route_on_two_calls_in_a_row():
         assert np.allclose(l1, l0, rtol=1e-5, atol=1e-6), name
         assert np.all(np.isfinite(w1)) and np.all(np.isfinite(l1))
         assert np.allclose(w1.sum(axis=1), wb.route_scale, rtol=1e-6)
+
+
+def test_route_noalloc_mid_batch_matches_the_oracle():
+    """At 600 tokens smoe_route runs on the tensor cores, the allocation-free router on the CUDA
+    cores (64-token x 96-expert tiles): checked against the fp64 oracle directly."""
+    w = synth.WORKLOADS["prefill"]
+    T = 600
+    cfg = smoe.config(w.H, w.E, w.k, w.I, w.Is, w.route_scale)
+    xh = synth.host_x_rows(w, np.arange(T))
+    x = torch.from_numpy(xh.view(np.int16)).cuda().view(torch.bfloat16)
+    wr, _ = synth.dev_router(w)
+    bias_h = synth.host_bias(w)
+    idx = torch.empty(T, w.k, dtype=torch.int32, device="cuda")
+    wt = torch.empty(T, w.k, dtype=torch.float32, device="cuda")
+    smoe.smoe_route_noalloc(cfg, x, T, wr, torch.from_numpy(bias_h).cuda(), idx, wt, None)
+    gi, gw = idx.cpu().numpy(), wt.cpu().numpy().astype(np.float64)
+    r = oracle.route(oracle.bf16_to_f64(xh), oracle.f32_to_f64(synth.host_w_router(w)), bias_h.astype(np.float64),
+                     w.k, w.route_scale)
+    for t in range(T):
+        ok, _ = selection_ok(r, t, tuple(sorted(gi[t].tolist())), w.k)
+        assert ok, f"token {t}"
+        if not r.near_tie[t]:
+            ref_w = dict(zip(r.idx[t].tolist(), r.w[t].tolist()))
+            assert np.allclose(gw[t], [ref_w[e] for e in gi[t].tolist()], rtol=1e-5, atol=0), f"token {t}"
 
 
 def test_route_noalloc_rejects_sizes_beyond_its_scratch():
