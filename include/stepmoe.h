@@ -102,10 +102,12 @@ SMOE_API smoe_status_t smoe_packed_weight_bytes(const smoe_config_t* cfg, size_t
  *   w_down        [E][H][I] bf16      routed down projections
  *   ws_gate, ws_up [Is][H] bf16, ws_down [H][Is] bf16   the shared expert
  *   packed        device buffer of smoe_packed_weight_bytes bytes, written here.
- * Packed layout: gate/up block [(E+1)][I/128][2][128][H] (for each 128-feature block,
- * 128 gate rows then the matching 128 up rows; group E = shared expert), followed by the
- * down block [(E+1)][H][I]. Source: the SwiGLU expert (paperlayer.ai summary, §B) with
- * moe_intermediate_size / share_expert_dim of the model card. Run once per layer. */
+ * Packed layout (tile-major: each tile the GEMMs load is contiguous): the gate/up block
+ * [(E+1)][I/128][H/64][256][64] (tile (g, mb, kb) = the 128 gate rows of features
+ * 128 mb .. 128 mb + 127, then the matching 128 up rows, over K columns 64 kb .. 64 kb + 63;
+ * group E = shared expert), followed by the down block [(E+1)][H/128][I/64][128][64].
+ * Source: the SwiGLU expert (paperlayer.ai summary, §B) with moe_intermediate_size /
+ * share_expert_dim of the model card. Run once per layer. */
 SMOE_API smoe_status_t smoe_pack_weights(const smoe_config_t* cfg, const smoe_bf16_t* w_gate, const smoe_bf16_t* w_up,
                                 const smoe_bf16_t* w_down, const smoe_bf16_t* ws_gate, const smoe_bf16_t* ws_up,
                                 const smoe_bf16_t* ws_down, void* packed, void* stream);

@@ -55,10 +55,6 @@ constexpr int kMaxStages = SMOE_MAX_STAGES;
 #define SMOE_PAIR_MIN_TILE 64    // CTA pairs for launches whose largest token tile is at least this
 #endif
 constexpr int kPairMinTile = SMOE_PAIR_MIN_TILE;
-#ifndef SMOE_PAIR_PREFETCH
-#define SMOE_PAIR_PREFETCH 0     // CTA pairs: L2 prefetch of the weight tile this many k-blocks ahead (0 = off)
-#endif
-constexpr int kPairPrefetch = SMOE_PAIR_PREFETCH;
 
 struct GemmMaps {
     CUtensorMap w;                  // weights [rows][K]: box {BK, 256 (gate/up) or 128 (down)}
@@ -137,6 +133,16 @@ __device__ __forceinline__ int tile_index(int nt) { return 31 - __clz(nt) - 4; }
 // M=128 and M=256 MMAs), at most the tile. A group of 228 rows loads a 256-row tile but runs
 // N=240 MMAs; the columns past N are never stored.
 __device__ __forceinline__ int mma_cols(int nvalid, int nt) { return min(nt, (nvalid + 15) & ~15); }
+
+// Packed expert weights are tile-major: weight block bi (R rows), K columns 64 kb .. 64 kb + 63
+// form one contiguous R x 64 tile, viewed by the tensor map as rows of a [*][64] matrix.
+// Coordinates (x, y) of the BK-wide K slice kg of block bi (K = the reduction length).
+template <int BK>
+__device__ __forceinline__ void weight_tile_xy(int bi, int kg, int K, int R, int& x, int& y) {
+    const int k0 = kg * BK;
+    x = k0 & 63;
+    y = (bi * (K / 64) + (k0 >> 6)) * R;
+}
 
 __device__ __forceinline__ Unit decode_unit(int u, const int32_t* prefix, const int32_t* offs, int E, int T,
                                             int nt_max) {
@@ -318,7 +324,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
             const int kb0 = (w.mb / MB) * KB;   // first k-block of this unit's K range
             w.mb %= MB;
-            const int a_row = DUAL ? (w.g * MB + w.mb) * 256 : w.g * p.n_out + w.mb * 128;
+            const int a_row = DUAL ? (w.g * MB + w.mb) * 256 : w.g * p.n_out + w.mb * 128;   // router: row-major
             const int b_row = (w.g < E ? offs[w.g] : p.shared_in_row) + w.nb * w.nt;
             const int ti = tile_index(w.nt);
             const bool gather = p.row_token != nullptr && w.g < E;
@@ -348,7 +354,13 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 const int b_k = p.k_wrap ? (kg % p.k_wrap) : kg;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(fb, tx);
-                    tma_load_2d(smem_u32(a_s), &maps.w, kg * BK, a_row, fb, pol_w);
+                    if (MODE == MODE_ROUTER) {
+                        tma_load_2d(smem_u32(a_s), &maps.w, kg * BK, a_row, fb, pol_w);
+                    } else {
+                        int wx, wy;
+                        weight_tile_xy<BK>(w.g * MB + w.mb, kg, p.K, C::A_ROWS, wx, wy);
+                        tma_load_2d(smem_u32(a_s), &maps.w, wx, wy, fb, pol_w);
+                    }
                     if (!gather) tma_load_2d(smem_u32(a_s + C::A_BYTES), bm, b_k * BK, b_row, fb, pol_a);
                 }
                 __syncwarp(pmask);
@@ -592,7 +604,7 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
         bool ok = true;
         for (int u = pair; ok && u < total; u += npairs) {
             const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);   // w.mb = 256-feature block
-            const int a_row = DUAL ? (w.g * MB + 2 * w.mb + (int)rank) * 256 : w.g * p.n_out + w.mb * 256 + (int)rank * 128;
+            const int a_blk = w.g * MB + 2 * w.mb + (int)rank;   // this CTA's 128-feature weight block
             // each CTA holds half of the MMA's N columns: the first CTA token rows 0..n/2-1 of the
             // tile, the second n/2..n-1 (its box of nt/2 rows may run past them; those rows are
             // never read)
@@ -602,26 +614,16 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
             const int ti = tile_index(w.nt);
             const CUtensorMap* bm = (w.g < E) ? &maps.act[ti] : &maps.sh[ti];
             const uint32_t tx = (uint32_t)(2 * (C::A_BYTES + half * BK * 2));
-            int next_a_row = -1;   // weight rows of this pair's next unit (prefetch target)
-            if (kPairPrefetch > 0 && u + npairs < total) {
-                const Unit nx = decode_unit(u + npairs, prefix, offs, E, p.T, p.nt_max);
-                next_a_row = DUAL ? (nx.g * MB + 2 * nx.mb + (int)rank) * 256 : nx.g * p.n_out + nx.mb * 256 + (int)rank * 128;
-            }
             for (int kb = 0; kb < KB; ++kb) {
                 if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag, true)) { ok = false; break; }
                 const uint32_t fb_local = smem_u32(&full[stage]);
                 const uint32_t fb_leader = mapa_shared(fb_local, 0);
                 if (rank == 0) mbar_arrive_expect_tx(fb_local, tx);
                 uint8_t* a_s = tiles + (size_t)stage * STAGE_B;
-                tma_load_2d_pair(smem_u32(a_s), &maps.w, kb * BK, a_row, fb_leader, pol_w);
+                int wx, wy;
+                weight_tile_xy<BK>(a_blk, kb, p.K, C::A_ROWS, wx, wy);
+                tma_load_2d_pair(smem_u32(a_s), &maps.w, wx, wy, fb_leader, pol_w);
                 tma_load_2d_pair(smem_u32(a_s + C::A_BYTES), bm, kb * BK, b_row, fb_leader, pol_a);
-                if (kPairPrefetch > 0) {
-                    const int kp = kb + kPairPrefetch;
-                    if (kp < KB)
-                        tma_prefetch_l2_2d(&maps.w, kp * BK, a_row);
-                    else if (next_a_row >= 0 && kp - KB < KB)
-                        tma_prefetch_l2_2d(&maps.w, (kp - KB) * BK, next_a_row);
-                }
                 armed |= 1u << stage;
                 armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                 if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -885,9 +887,10 @@ cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const u
     bool ok_act = gather ? make_map(&m1.act[0], x, (uint64_t)T, H, 1, BK) : act_maps(m1.act, x_perm, (uint64_t)routed, H);
     if (gather)
         for (int i = 1; i < kNumTiles; ++i) m1.act[i] = m1.act[0];
-    if (!ok_act || !make_map(&m1.w, wgu, (uint64_t)(E + 1) * 2 * I, H, 256, BK) ||
+    // packed weights, tile-major: viewed as [rows][64] with 256-row (gate/up) / 128-row (down) tiles
+    if (!ok_act || !make_map(&m1.w, wgu, (uint64_t)(E + 1) * 2 * I * (H / 64), 64, 256, BK) ||
         !act_maps(m1.sh, x, (uint64_t)T, H) ||
-        !make_map(&m2.w, wdn, (uint64_t)(E + 1) * H, I, 128, BK) ||
+        !make_map(&m2.w, wdn, (uint64_t)(E + 1) * H * (I / 64), 64, 128, BK) ||
         !act_maps(m2.act, h, (uint64_t)(routed + T), I))
         return cudaErrorNotSupported;
     for (int i = 0; i < kNumTiles; ++i) m2.sh[i] = m2.act[i];

@@ -1,7 +1,11 @@
 // Weight packing for the expert GEMMs (a one-time layout transform, not part of a step).
-//   gate/up block: [(E+1)][I/128][2][128][H]  — per 128-feature block, the 128 gate rows then
-//                  the 128 matching up rows, so one 256-row TMA box feeds both MMAs;
-//   down block:    [(E+1)][H][I]              — routed experts then the shared expert.
+// Tile-major: every weight tile one TMA load brings into shared memory (R rows x 64 K columns,
+// 128-byte rows) is one contiguous block in HBM, so each load streams whole DRAM pages.
+//   gate/up: [(E+1)][I/128][H/64][256][64] — tile (g, mb, kb): rows 0-127 the gate rows of
+//            features 128 mb .. 128 mb + 127, rows 128-255 the matching up rows, columns
+//            64 kb .. 64 kb + 63 of K = H; one 256-row box feeds both MMAs;
+//   down:    [(E+1)][H/128][I/64][128][64]  — tile (g, mb, kb): rows 128 mb .. + 127 of W_d,
+//            columns 64 kb .. + 63 of K = I.
 // Group E is the shared expert (Step 3.5 Flash summary, hyper.ai, section "方法": one shared
 // expert beside the routed ones; model card field share_expert_dim 1280).
 #include "common.cuh"
@@ -11,41 +15,50 @@ namespace smoe {
 
 namespace {
 
-// One warp per destination row; rows are copied with 16-byte vectors.
+// One thread per 16-byte chunk of a destination tile row (8 chunks = the row's 64 elements).
+// Destination tile row tr = ((bi * KT + kb) * R + r) with bi = g * MB + mb; the source row of
+// (g, mb, r) comes from src_row(), its columns 64 kb .. 64 kb + 63.
+template <typename SrcRow>
+__device__ __forceinline__ void pack_tiles(int64_t ntr, int R, int KT, int MB, int K, uint16_t* __restrict__ dst,
+                                           SrcRow src_row) {
+    const int64_t nchunks = ntr * 8;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nchunks; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t tr = i >> 3;
+        const int ch = (int)(i & 7);
+        const int r = (int)(tr % R);
+        const int64_t tile = tr / R;
+        const int kb = (int)(tile % KT);
+        const int64_t bi = tile / KT;
+        const int g = (int)(bi / MB), mb = (int)(bi % MB);
+        const uint16_t* src = src_row(g, mb, r);
+        reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<const uint4*>(src + (size_t)kb * 64 + ch * 8);
+    }
+    (void)K;
+}
+
 __global__ void __launch_bounds__(256) pack_gateup_kernel(const uint16_t* __restrict__ wg,
                                                           const uint16_t* __restrict__ wu,
                                                           const uint16_t* __restrict__ sg,
                                                           const uint16_t* __restrict__ su, int E, int I, int H,
                                                           uint16_t* __restrict__ dst) {
-    const int64_t nrows = (int64_t)(E + 1) * 2 * I;
-    const int lane = threadIdx.x & 31;
-    const int vec = H / 8;
-    for (int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); r < nrows; r += (int64_t)gridDim.x * 8) {
-        const int g = (int)(r / (2 * I));
-        const int rr = (int)(r % (2 * I));
-        const int mb = rr / 256, w = rr % 256;
-        const int feat = mb * 128 + (w & 127);
-        const bool up = w >= 128;
-        const uint16_t* src = (g < E) ? ((up ? wu : wg) + ((size_t)g * I + feat) * H) : ((up ? su : sg) + (size_t)feat * H);
-        const uint4* s4 = reinterpret_cast<const uint4*>(src);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)r * H);
-        for (int c = lane; c < vec; c += 32) d4[c] = s4[c];
-    }
+    const int MB = I / 128, KT = H / 64;
+    const int64_t ntr = (int64_t)(E + 1) * MB * KT * 256;
+    pack_tiles(ntr, 256, KT, MB, H, dst, [&](int g, int mb, int r) {
+        const int feat = mb * 128 + (r & 127);
+        const bool up = r >= 128;
+        return (g < E) ? ((up ? wu : wg) + ((size_t)g * I + feat) * H) : ((up ? su : sg) + (size_t)feat * H);
+    });
 }
 
 __global__ void __launch_bounds__(256) pack_down_kernel(const uint16_t* __restrict__ wd,
                                                         const uint16_t* __restrict__ sd, int E, int I, int H,
                                                         uint16_t* __restrict__ dst) {
-    const int64_t nrows = (int64_t)(E + 1) * H;
-    const int lane = threadIdx.x & 31;
-    const int vec = I / 8;
-    for (int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); r < nrows; r += (int64_t)gridDim.x * 8) {
-        const int g = (int)(r / H);
-        const uint16_t* src = (g < E) ? (wd + (size_t)r * I) : (sd + (size_t)(r - (int64_t)E * H) * I);
-        const uint4* s4 = reinterpret_cast<const uint4*>(src);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)r * I);
-        for (int c = lane; c < vec; c += 32) d4[c] = s4[c];
-    }
+    const int MB = H / 128, KT = I / 64;
+    const int64_t ntr = (int64_t)(E + 1) * MB * KT * 128;
+    pack_tiles(ntr, 128, KT, MB, I, dst, [&](int g, int mb, int r) {
+        const int row = mb * 128 + r;
+        return (g < E) ? (wd + ((size_t)g * H + row) * I) : (sd + (size_t)row * I);
+    });
 }
 
 }  // namespace
