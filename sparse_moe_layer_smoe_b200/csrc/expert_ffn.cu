@@ -17,8 +17,9 @@
 // Token tile per group: the smallest power of two >= the group's row count, between 16 and a
 // launch-wide maximum NT_MAX (so an expert with 2 tokens runs N=16 MMAs while a hot expert with
 // 1000 tokens runs N=256 tiles). One TMA tensor map per tile height loads exactly that box.
-// Work unit = (group, 128-feature block mb, token tile nb), enumerated group-major, then mb,
-// then nb; CTA i takes units i, i + grid, ... (static persistent schedule, grid = #SMs).
+// Work unit = (token tile (group, nb), 128-feature block mb). The token tiles are sorted by the
+// MMA columns they run (largest first) and the units dealt to the CTAs in snake order (static
+// persistent schedule, grid = #SMs): see the work table below.
 //
 // Roles (192 threads): warp 0 lane 0 issues TMA loads into an S-stage ring of BK-wide K slices
 // (BK = 64: 128-byte swizzled rows; the ring fills the 227 KB of shared memory);
@@ -84,6 +85,7 @@ struct GemmParams {
     uint16_t* out;            // [*, out_ld] bf16 (gate/up, down)
     float* out_f32;           // [*, out_ld] fp32 (router)
     int32_t* err;
+    int max_tiles;            // capacity of the token-tile table in shared memory
 };
 
 // What a launch computes: the down projection, the fused gate/up + SiLU*mul, or router logits.
@@ -103,12 +105,19 @@ __host__ __device__ inline int stage_bytes(bool dual, int bk, int nt_max) {
     return (dual ? 256 : 128) * bk * 2 + nt_max * bk * 2;
 }
 
-__host__ __device__ inline size_t gemm_smem_bytes(int stages, int stage_b, int E) {
+// Upper bound on the token tiles of a launch: a group of r rows has one tile if r <= nt_max,
+// else ceil(r / nt_max) <= r / nt_max + 1, and the rows of all groups add up to at most
+// routed_rows + T.
+__host__ __device__ inline int max_token_tiles(int E, int routed_rows, int T, int nt_max) {
+    return E + 2 + (routed_rows + T) / nt_max;
+}
+
+__host__ __device__ inline size_t gemm_smem_bytes(int stages, int stage_b, int E, int max_tiles) {
     size_t b = 1024;                                       // alignment slack
     b += (size_t)stages * stage_b;
     b += sizeof(uint64_t) * (2 * (size_t)stages + 5);      // full, empty, tfull[2], tempty[2], drain
-    b += 16;                                               // tmem slot, abort flag
-    b += sizeof(int32_t) * (2 * (size_t)E + 3);            // prefix[E+2], offs[E+1]
+    b += 16;                                               // tmem slot, abort flag, tile count
+    b += sizeof(int32_t) * ((size_t)max_tiles + E + 1);    // tiles[max_tiles], offs[E+1]
     return b;
 }
 
@@ -144,19 +153,76 @@ __device__ __forceinline__ void weight_tile_xy(int bi, int kg, int K, int R, int
     y = (bi * (K / 64) + (k0 >> 6)) * R;
 }
 
-__device__ __forceinline__ Unit decode_unit(int u, const int32_t* prefix, const int32_t* offs, int E, int T,
-                                            int nt_max) {
-    int lo = 0, hi = E;   // find g with prefix[g] <= u < prefix[g+1]
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (prefix[mid] <= u) lo = mid; else hi = mid - 1;
+// Work table. A token tile is (group g, tile nb) of nt rows; a unit is (tile, feature block
+// [, K range]), units_per_tile of them per tile, numbered tile-major, tiles in group order. The
+// units are dealt to the W workers (CTAs or CTA pairs) in snake order: round i gives unit
+// i*W + w to worker w on even rounds and i*W + W-1-w on odd ones, which evens out the work per
+// worker when unit costs vary (skewed batches); the units of one tile (the same token rows)
+// run at the same time on neighbouring workers, which share those rows in L2. (Measured: listing
+// the tiles sorted by cost, largest first, made skewed batches 2-3% slower than group order.)
+__device__ __forceinline__ Unit decode_unit(int u, int units_per_tile, const int32_t* tiles, const int32_t* offs,
+                                            int E, int T, int nt_max) {
+    const int t = tiles[u / units_per_tile];
+    const int g = t >> 20;
+    const int nt = group_tile(group_rows(g, E, T, offs), nt_max);
+    return Unit{g, u % units_per_tile, t & 0xFFFFF, nt};
+}
+
+// Unit of round i for worker w of W (snake order), or -1 when it lies past the last unit.
+__device__ __forceinline__ int snake_unit(int i, int w, int W, int total) {
+    const int u = i * W + ((i & 1) ? W - 1 - w : w);
+    return u < total ? u : -1;
+}
+
+// One warp: validate the offsets into offs[] (corrupt offsets: no routed work, the error word
+// set), then list the token tiles in tiles[] (entry g << 20 | nb) in group order. Returns the
+// tile count. Lane l owns a contiguous range of groups and one warp scan places its tiles:
+// every CTA of the launch builds the same table.
+__device__ int build_tile_table(const int32_t* offsets, int E, int T, int routed_rows, int nt_max, int max_tiles,
+                                int32_t* offs, int32_t* tiles, int32_t* err) {
+    const int lane = threadIdx.x & 31;
+    bool bad = false;
+    for (int i = lane; i <= E; i += 32) {
+        int v = (offsets != nullptr) ? offsets[i] : 0;
+        if (v < 0 || v > routed_rows) { bad = true; v = 0; }
+        offs[i] = v;
     }
-    const int g = lo;
-    const int rows = group_rows(g, E, T, offs);
-    const int nt = group_tile(rows, nt_max);
-    const int nblk = (rows + nt - 1) / nt;
-    const int local = u - prefix[g];
-    return Unit{g, local / nblk, local % nblk, nt};
+    __syncwarp();
+    for (int i = lane; i < E; i += 32)
+        if (offs[i + 1] < offs[i]) bad = true;
+    if (__any_sync(0xFFFFFFFFu, bad)) {
+        for (int i = lane; i <= E; i += 32) offs[i] = 0;
+        if (lane == 0) record_error(err, SMOE_ERR_DEVICE);
+    }
+    __syncwarp();
+    const int ngroups = E + 1;
+    const int chunk = (ngroups + 31) / 32;
+    const int g0 = min(lane * chunk, ngroups), g1 = min(g0 + chunk, ngroups);
+    auto tiles_of = [&](int g) {
+        const int rows = group_rows(g, E, T, offs);
+        const int nt = group_tile(rows, nt_max);
+        return (rows + nt - 1) / nt;
+    };
+    int local = 0;
+    for (int g = g0; g < g1; ++g) local += tiles_of(g);
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off) incl += n;
+    }
+    int pos = incl - local;
+    for (int g = g0; g < g1; ++g) {
+        const int nblk = tiles_of(g);
+        for (int nb = 0; nb < nblk; ++nb, ++pos)
+            if (pos < max_tiles) tiles[pos] = (g << 20) | nb;
+    }
+    int n = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    if (n > max_tiles) {   // cannot happen for validated offsets; never read past the table
+        if (lane == 0) record_error(err, SMOE_ERR_DEVICE);
+        n = 0;
+    }
+    return n;
 }
 
 // Epilogue, part 1: drain this thread's accumulator row (one output feature, up to 256 token
@@ -227,8 +293,9 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     uint64_t* drain = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int32_t* prefix = reinterpret_cast<int32_t*>(tmem_slot + 4);   // [E+2]
-    int32_t* offs = prefix + (p.E + 2);                              // [E+1]
+    int* ntiles_slot = reinterpret_cast<int*>(tmem_slot + 2);
+    int32_t* ttab = reinterpret_cast<int32_t*>(tmem_slot + 4);     // token tiles [max_tiles]
+    int32_t* offs = ttab + p.max_tiles;                              // [E+1]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
@@ -261,50 +328,15 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             }
     }
     if (warp == 2) {
-        // group table: offsets (validated), then units per group and their exclusive prefix
-        bool bad = false;
-        for (int i = lane; i <= E; i += 32) {
-            int v = (p.offsets != nullptr) ? p.offsets[i] : 0;
-            if (v < 0 || v > p.routed_rows) { bad = true; v = 0; }
-            offs[i] = v;
-        }
-        __syncwarp();
-        for (int i = lane; i < E; i += 32)
-            if (offs[i + 1] < offs[i]) bad = true;
-        if (__any_sync(0xFFFFFFFFu, bad)) {
-            // corrupt offsets: run no routed work (shared expert only)
-            for (int i = lane; i <= E; i += 32) offs[i] = 0;
-            if (lane == 0) record_error(p.err, SMOE_ERR_DEVICE);
-        }
-        __syncwarp();
-        const int ngroups = E + 1;
-        const int chunk = (ngroups + 31) / 32;
-        const int g0 = min(lane * chunk, ngroups), g1 = min(g0 + chunk, ngroups);
-        auto units_of = [&](int g) {
-            const int rows = group_rows(g, E, p.T, offs);
-            const int nt = group_tile(rows, p.nt_max);
-            return ((rows + nt - 1) / nt) * MB * p.ksplit;
-        };
-        int local = 0;
-        for (int g = g0; g < g1; ++g) local += units_of(g);
-        int incl = local;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int n = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-            if (lane >= off) incl += n;
-        }
-        int run = incl - local;
-        for (int g = g0; g < g1; ++g) {
-            prefix[g] = run;
-            run += units_of(g);
-        }
-        if (lane == 31) prefix[E + 1] = incl;
+        const int n = build_tile_table(p.offsets, E, p.T, p.routed_rows, p.nt_max, p.max_tiles, offs, ttab, p.err);
+        if (lane == 0) *ntiles_slot = n;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int total = prefix[E + 1];
+    const int upt = MB * p.ksplit;   // units per token tile
+    const int total = *ntiles_slot * upt;
 
     // gather mode (row_token set) uses all 32 producer lanes; otherwise lane 0 alone, so the
     // stage refill path carries no warp-wide synchronisation
@@ -320,8 +352,10 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         int stage = 0;
         uint32_t phase = 0, armed = 0, armed_par = 0;
         bool ok = true;
-        for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
-            Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
+        for (int i = 0; ok && i * (int)gridDim.x < total; ++i) {
+            const int u = snake_unit(i, blockIdx.x, gridDim.x, total);
+            if (u < 0) continue;
+            Unit w = decode_unit(u, upt, ttab, offs, E, p.T, p.nt_max);
             const int kb0 = (w.mb / MB) * KB;   // first k-block of this unit's K range
             w.mb %= MB;
             const int a_row = DUAL ? (w.g * MB + w.mb) * 256 : w.g * p.n_out + w.mb * 128;   // router: row-major
@@ -389,8 +423,10 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         int stage = 0, acc = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
-        for (int u = blockIdx.x; ok && u < total; u += gridDim.x) {
-            const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
+        for (int i = 0; ok && i * (int)gridDim.x < total; ++i) {
+            const int u = snake_unit(i, blockIdx.x, gridDim.x, total);
+            if (u < 0) continue;
+            const Unit w = decode_unit(u, upt, ttab, offs, E, p.T, p.nt_max);
             const int n_mma = mma_cols(group_rows(w.g, E, p.T, offs) - w.nb * w.nt, w.nt);
             const uint32_t idesc = idesc0 | ((uint32_t)(n_mma >> 3) << 17);
             if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, p.err, abort_flag, true)) break;
@@ -431,8 +467,10 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         const int row = q * 32 + lane;     // accumulator row = output feature within the block
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int u = blockIdx.x; u < total; u += gridDim.x) {
-            Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
+        for (int i = 0; i * (int)gridDim.x < total; ++i) {
+            const int u = snake_unit(i, blockIdx.x, gridDim.x, total);
+            if (u < 0) continue;
+            Unit w = decode_unit(u, upt, ttab, offs, E, p.T, p.nt_max);
             const int kp = w.mb / MB;   // K range of this unit (partial output kp)
             w.mb %= MB;
             const int rows = group_rows(w.g, E, p.T, offs);
@@ -488,8 +526,8 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
 // the token rows (nt/2); one 256-row MMA issued by the first CTA reads both CTAs' shared memory
 // and accumulates into both CTAs' TMEM (128 rows each). Per SM this moves 25-30% fewer operand
 // bytes through shared memory per MMA than the single-CTA kernel, whose token tile every SM
-// loads in full. Work unit = (group, 256-feature block, token tile); pair p takes units p,
-// p + pairs, ...
+// loads in full. Work unit = (token tile, 256-feature block), dealt to the pairs in the same
+// cost-sorted snake order as the single-CTA kernel's units.
 //
 // Signals: both CTAs' loads complete on the first CTA's stage barrier (it arms the expected
 // bytes of both); the first CTA's MMA thread commits stage-free and accumulator-ready to each
@@ -515,8 +553,9 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
     uint64_t* drain = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int32_t* prefix = reinterpret_cast<int32_t*>(tmem_slot + 4);   // [E+2]
-    int32_t* offs = prefix + (p.E + 2);                              // [E+1]
+    int* ntiles_slot = reinterpret_cast<int*>(tmem_slot + 2);
+    int32_t* ttab = reinterpret_cast<int32_t*>(tmem_slot + 4);     // token tiles [max_tiles]
+    int32_t* offs = ttab + p.max_tiles;                              // [E+1]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -552,48 +591,14 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
             }
     }
     if (warp == 2) {
-        bool bad = false;
-        for (int i = lane; i <= E; i += 32) {
-            int v = (p.offsets != nullptr) ? p.offsets[i] : 0;
-            if (v < 0 || v > p.routed_rows) { bad = true; v = 0; }
-            offs[i] = v;
-        }
-        __syncwarp();
-        for (int i = lane; i < E; i += 32)
-            if (offs[i + 1] < offs[i]) bad = true;
-        if (__any_sync(0xFFFFFFFFu, bad)) {
-            for (int i = lane; i <= E; i += 32) offs[i] = 0;
-            if (lane == 0) record_error(p.err, SMOE_ERR_DEVICE);
-        }
-        __syncwarp();
-        const int ngroups = E + 1;
-        const int chunk = (ngroups + 31) / 32;
-        const int g0 = min(lane * chunk, ngroups), g1 = min(g0 + chunk, ngroups);
-        auto units_of = [&](int g) {
-            const int rows = group_rows(g, E, p.T, offs);
-            const int nt = group_tile(rows, p.nt_max);
-            return ((rows + nt - 1) / nt) * MBP;
-        };
-        int local = 0;
-        for (int g = g0; g < g1; ++g) local += units_of(g);
-        int incl = local;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int n = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-            if (lane >= off) incl += n;
-        }
-        int run = incl - local;
-        for (int g = g0; g < g1; ++g) {
-            prefix[g] = run;
-            run += units_of(g);
-        }
-        if (lane == 31) prefix[E + 1] = incl;
+        const int n = build_tile_table(p.offsets, E, p.T, p.routed_rows, p.nt_max, p.max_tiles, offs, ttab, p.err);
+        if (lane == 0) *ntiles_slot = n;
     }
     tc_fence_before();
     cluster_sync();   // barrier inits and TMEM allocation visible to both CTAs
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int total = prefix[E + 1];
+    const int total = *ntiles_slot * MBP;   // units: (token tile, 256-feature block)
 
     if (warp == 0 && lane == 0) {
         // ---------------------------------------------------------------- TMA producer (both CTAs)
@@ -602,8 +607,10 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
         int stage = 0;
         uint32_t phase = 0, armed = 0, armed_par = 0;
         bool ok = true;
-        for (int u = pair; ok && u < total; u += npairs) {
-            const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);   // w.mb = 256-feature block
+        for (int i = 0; ok && i * npairs < total; ++i) {
+            const int u = snake_unit(i, pair, npairs, total);
+            if (u < 0) continue;
+            const Unit w = decode_unit(u, MBP, ttab, offs, E, p.T, p.nt_max);   // w.mb = 256-feature block
             const int a_blk = w.g * MB + 2 * w.mb + (int)rank;   // this CTA's 128-feature weight block
             // each CTA holds half of the MMA's N columns: the first CTA token rows 0..n/2-1 of the
             // tile, the second n/2..n-1 (its box of nt/2 rows may run past them; those rows are
@@ -641,8 +648,10 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
         int stage = 0, acc = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
-        for (int u = pair; ok && u < total; u += npairs) {
-            const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
+        for (int i = 0; ok && i * npairs < total; ++i) {
+            const int u = snake_unit(i, pair, npairs, total);
+            if (u < 0) continue;
+            const Unit w = decode_unit(u, MBP, ttab, offs, E, p.T, p.nt_max);
             const int n_mma = mma_cols(group_rows(w.g, E, p.T, offs) - w.nb * w.nt, w.nt);
             const uint32_t idesc = idesc0 | ((uint32_t)(n_mma >> 3) << 17);
             if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, p.err, abort_flag, true)) break;
@@ -686,8 +695,10 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
         const int row = q * 32 + lane;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int u = pair; u < total; u += npairs) {
-            const Unit w = decode_unit(u, prefix, offs, E, p.T, p.nt_max);
+        for (int i = 0; i * npairs < total; ++i) {
+            const int u = snake_unit(i, pair, npairs, total);
+            if (u < 0) continue;
+            const Unit w = decode_unit(u, MBP, ttab, offs, E, p.T, p.nt_max);
             const int rows = group_rows(w.g, E, p.T, offs);
             const int out_base = (w.g < E ? offs[w.g] : p.shared_out_row) + w.nb * w.nt;
             const int nvalid = min(w.nt, rows - w.nb * w.nt);
@@ -788,12 +799,14 @@ cudaError_t run_gemm(const GemmMaps& maps, GemmParams p, int grid, cudaStream_t 
     constexpr int BK = SMOE_GEMM_BK;
     constexpr bool DUAL = MODE == MODE_GATEUP;
     const int sb = stage_bytes(DUAL, BK, p.nt_max);
-    const size_t fixed = gemm_smem_bytes(0, sb, p.E) + 2 * sizeof(uint64_t) * kMaxStages;
+    p.max_tiles = max_token_tiles(p.E, p.routed_rows, p.T, p.nt_max);
+    const size_t fixed = gemm_smem_bytes(0, sb, p.E, p.max_tiles) + 2 * sizeof(uint64_t) * kMaxStages;
+    if (fixed >= (size_t)max_dynamic_smem()) return cudaErrorInvalidConfiguration;
     int stages = (int)((max_dynamic_smem() - fixed) / sb);
     if (stages > kMaxStages) stages = kMaxStages;
     if (stages < 2) return cudaErrorInvalidConfiguration;
     p.stages = stages;
-    const size_t smem = gemm_smem_bytes(stages, sb, p.E);
+    const size_t smem = gemm_smem_bytes(stages, sb, p.E, p.max_tiles);
     cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
@@ -822,12 +835,14 @@ cudaError_t run_gemm_pair(const GemmMaps& maps, GemmParams p, int num_sms, cudaS
     constexpr int BK = SMOE_GEMM_BK;
     constexpr bool DUAL = MODE == MODE_GATEUP;
     const int sb = (DUAL ? 256 : 128) * BK * 2 + (p.nt_max / 2) * BK * 2;
-    const size_t fixed = gemm_smem_bytes(0, sb, p.E) + 2 * sizeof(uint64_t) * kMaxStages;
+    p.max_tiles = max_token_tiles(p.E, p.routed_rows, p.T, p.nt_max);
+    const size_t fixed = gemm_smem_bytes(0, sb, p.E, p.max_tiles) + 2 * sizeof(uint64_t) * kMaxStages;
+    if (fixed >= (size_t)max_dynamic_smem()) return cudaErrorInvalidConfiguration;
     int stages = (int)((max_dynamic_smem() - fixed) / sb);
     if (stages > kMaxStages) stages = kMaxStages;
     if (stages < 2) return cudaErrorInvalidConfiguration;
     p.stages = stages;
-    const size_t smem = gemm_smem_bytes(stages, sb, p.E);
+    const size_t smem = gemm_smem_bytes(stages, sb, p.E, p.max_tiles);
     auto kern = expert_gemm_pair_kernel<MODE, BK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
