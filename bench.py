@@ -49,6 +49,7 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=4)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--diag", action="store_true", help="time smoe_forward_diag (layer + monitoring outputs)")
     return p.parse_args(argv)
 
 
@@ -249,6 +250,7 @@ def run_reference(args):
 def workload_config(w):
     return {"workload": w.name, "T": w.T, "hidden": w.H, "experts": w.E, "top_k": w.k, "inter": w.I,
             "shared_inter": w.Is, "route_scale": w.route_scale, "bias": w.bias, "spike_rows": w.spike_rows,
+            "swiglu_limit": w.swiglu_limit, "swiglu_limit_shared": w.swiglu_limit_shared,
             "parallelism": "replicas",
             "l2": "inputs larger than L2: every step streams the active experts' bf16 weights (GBs) from HBM"}
 
@@ -264,7 +266,7 @@ def run_ours(args):
     init_dist(world, "nccl")
     dev = torch.device("cuda", local)
     w = synth.WORKLOADS[args.workload]
-    cfg = smoe.config(w.H, w.E, w.k, w.I, w.Is, w.route_scale)
+    cfg = smoe.config(w.H, w.E, w.k, w.I, w.Is, w.route_scale, w.swiglu_limit, w.swiglu_limit_shared)
     T = w.T
 
     x = synth.dev_x(w, device=dev)
@@ -277,6 +279,13 @@ def run_ours(args):
     ws = smoe.workspace(cfg, T, device=dev)
     out = torch.empty(T, w.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
+    diag = smoe.diag_buffers(cfg, T, device=dev) if args.diag else None
+
+    def forward(x_):
+        if diag is None:
+            smoe.smoe_forward(cfg, x_, T, wr, bias, packed, out, ws)
+        else:
+            smoe.smoe_forward_diag(cfg, x_, T, wr, bias, packed, out, diag, ws)
 
     # routing statistics of this batch (for the algorithmic byte count): experts touched
     idx = torch.empty(T, w.k, dtype=torch.int32, device=dev)
@@ -289,7 +298,7 @@ def run_ours(args):
 
     # ---- device-resident timing (value)
     for _ in range(args.warmup):
-        smoe.smoe_forward(cfg, x, T, wr, bias, packed, out, ws)
+        forward(x)
     torch.cuda.synchronize()
     launches_per_step = smoe.smoe_last_launch_count()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -299,7 +308,7 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         ev0.record(stream)
         for _ in range(args.steps):
-            smoe.smoe_forward(cfg, x, T, wr, bias, packed, out, ws)
+            forward(x)
         ev1.record(stream)
         torch.cuda.synchronize()
     ktimes = smoe.smoe_timing_end()
@@ -317,7 +326,7 @@ def run_ours(args):
 
     def e2e_step():
         x_in.copy_(x_host, non_blocking=True)
-        smoe.smoe_forward(cfg, x_in, T, wr, bias, packed, out, ws)
+        forward(x_in)
         out_host.copy_(out, non_blocking=True)
         stream.synchronize()
 
@@ -366,7 +375,8 @@ def run_ours(args):
 
     line = {"metric": METRIC, "value": world * T / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w),
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {**workload_config(w), **({"diag": True} if args.diag else {})},
             "layer": {"hbm_gbs": layer_bytes / (ms / 1e3) / 1e9, "tflops": layer_flops / (ms / 1e3) / 1e12,
                       "experts_touched": touched, "algorithmic_bytes": layer_bytes},
             "kernels_ms_per_step": {n: t / args.steps for n, (_, t) in sorted(ktimes.items(), key=lambda kv: -kv[1][1])},

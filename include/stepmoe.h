@@ -176,6 +176,44 @@ SMOE_API smoe_status_t smoe_forward(const smoe_config_t* cfg, const smoe_bf16_t*
                            const float* bias, const void* packed, smoe_bf16_t* out, void* ws, size_t ws_bytes,
                            void* stream);
 
+/* Monitoring outputs of one layer step (smoe_forward_diag), after the Step 3.5 Flash
+ * summary (paperlayer.ai): §4.1.2 monitors per-expert activation norms (a falling
+ * minimum-to-median ratio warns of expert death), §4.1.3 reads localized activation blow-up
+ * from the maximum-to-median activation-norm ratio, §5.2.1 uses routing confidence as a
+ * stability proxy. The pages define none of these numerically; the readings here:
+ *   expert norm   ||F_e(x_t)||_2, the L2 norm of routed expert e's output row for token t
+ *                 (the bf16 row the layer combines, before its routing weight);
+ *   confidence    of token t: the mean of its k selected (unbiased) sigmoid scores.
+ * All pointers are caller-owned device arrays, 16-byte aligned, written on the stream. */
+typedef struct {
+    int32_t* expert_count;      /* [E] tokens routed to expert e */
+    float* expert_norm_mean;    /* [E] mean expert norm over those tokens (0 when none) */
+    float* expert_norm_max;     /* [E] largest expert norm over those tokens (0 when none) */
+    float* token_confidence;    /* [T] routing confidence of each token */
+    float* summary;             /* [SMOE_DIAG_SUMMARY] the layer summary, indexed below */
+} smoe_diag_t;
+
+enum {
+    SMOE_DIAG_ACTIVE_EXPERTS = 0,   /* experts that received at least one token */
+    SMOE_DIAG_NORM_MEDIAN,          /* median of expert_norm_mean over those experts (mean of the
+                                       two middle values for an even count) */
+    SMOE_DIAG_NORM_MAX_TO_MEDIAN,   /* their largest expert_norm_mean / the median (0 if median 0) */
+    SMOE_DIAG_NORM_MIN_TO_MEDIAN,   /* their smallest expert_norm_mean / the median (0 if median 0) */
+    SMOE_DIAG_CONF_MEAN,            /* mean token confidence */
+    SMOE_DIAG_CONF_MIN,             /* smallest token confidence */
+    SMOE_DIAG_LOAD_MAX_TO_MEAN,     /* largest expert_count / (T * k / E) */
+    SMOE_DIAG_NORM_PEAK,            /* largest expert_norm_max */
+    SMOE_DIAG_SUMMARY               /* number of summary entries */
+};
+
+/* smoe_forward plus the monitoring outputs above (diag must be non-NULL, every array set).
+ * Same workspace as smoe_forward; the extra work is a sum of squares per routed row inside
+ * the combine kernel, the confidence store in the top-k kernel and one single-CTA kernel.
+ * Every output is deterministic. Returns SMOE_ERR_INVALID_ARG for a NULL or misaligned array. */
+SMOE_API smoe_status_t smoe_forward_diag(const smoe_config_t* cfg, const smoe_bf16_t* x, int64_t T,
+                                const float* w_router, const float* bias, const void* packed, smoe_bf16_t* out,
+                                const smoe_diag_t* diag, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronise `stream` and read the workspace's device error word into *code
  * (SMOE_OK when no kernel recorded an error). */
 SMOE_API smoe_status_t smoe_get_device_error(const void* ws, int32_t* code, void* stream);
@@ -191,7 +229,7 @@ SMOE_API int32_t smoe_last_launch_count(void);
 typedef struct {
     char name[32];       /* kernel: router_logits, router_topk, permute_hist, permute_scan,
                             permute_scatter, gather_rows, expert_gateup, expert_down, combine,
-                            pack_gateup, pack_down */
+                            pack_gateup, pack_down, router_split, router_gemm, diag */
     int32_t launches;    /* launches recorded */
     float total_ms;      /* summed event-to-event time of those launches */
 } smoe_kernel_time_t;

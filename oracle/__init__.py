@@ -4,10 +4,11 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline / r
 leg may import this package. The CUDA library never imports it and shares no code with it.
 Parity status of each function (what pins it) is stated in ``tests/test_oracle_pins.py``.
 """
+from .diag import SUMMARY_FIELDS, Diagnostics, diagnostics, expert_output_norms, summarise
 from .moe import (NEAR_TIE_EPS, Route, bf16_to_f64, combine, f32_to_f64, moe_dense_masked, moe_given_selection,
                   moe_sparse, normalise, permute, route, router_logits, select_topk, sigmoid, silu, swiglu_ffn,
                   swiglu_hidden, valid_selections)
 
-__all__ = ["NEAR_TIE_EPS", "Route", "bf16_to_f64", "combine", "f32_to_f64", "moe_dense_masked",
-           "moe_given_selection", "moe_sparse", "normalise", "permute", "route", "router_logits", "select_topk",
+__all__ = ["SUMMARY_FIELDS", "Diagnostics", "diagnostics", "expert_output_norms", "summarise", "NEAR_TIE_EPS",
+           "Route", "bf16_to_f64", "combine", "f32_to_f64", "moe_dense_masked", "moe_given_selection", "moe_sparse", "normalise", "permute", "route", "router_logits", "select_topk",
            "sigmoid", "silu", "swiglu_ffn", "swiglu_hidden", "valid_selections"]

@@ -43,6 +43,19 @@ class SmoeKernelTime(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int32), ("total_ms", ctypes.c_float)]
 
 
+class SmoeDiag(ctypes.Structure):
+    """smoe_diag_t: device pointers of the monitoring outputs (see include/stepmoe.h)."""
+    _fields_ = [("expert_count", ctypes.c_void_p), ("expert_norm_mean", ctypes.c_void_p),
+                ("expert_norm_max", ctypes.c_void_p), ("token_confidence", ctypes.c_void_p),
+                ("summary", ctypes.c_void_p)]
+
+
+# indices into smoe_diag_t.summary
+(SMOE_DIAG_ACTIVE_EXPERTS, SMOE_DIAG_NORM_MEDIAN, SMOE_DIAG_NORM_MAX_TO_MEDIAN, SMOE_DIAG_NORM_MIN_TO_MEDIAN,
+ SMOE_DIAG_CONF_MEAN, SMOE_DIAG_CONF_MIN, SMOE_DIAG_LOAD_MAX_TO_MEAN, SMOE_DIAG_NORM_PEAK, SMOE_DIAG_SUMMARY) = range(9)
+DIAG_FIELDS = ("expert_count", "expert_norm_mean", "expert_norm_max", "token_confidence", "summary")
+
+
 _vp, _i64, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
 _cfgp = ctypes.POINTER(SmoeConfig)
 _SIGS = {
@@ -57,6 +70,8 @@ _SIGS = {
     "smoe_expert_ffn": ([_cfgp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "smoe_combine": ([_cfgp, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _vp], ctypes.c_int),
     "smoe_forward": ([_cfgp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "smoe_forward_diag": ([_cfgp, _vp, _i64, _vp, _vp, _vp, _vp, ctypes.POINTER(SmoeDiag), _vp, _sz, _vp],
+                          ctypes.c_int),
     "smoe_get_device_error": ([_vp, ctypes.POINTER(ctypes.c_int32), _vp], ctypes.c_int),
     "smoe_clear_device_error": ([_vp, _vp], ctypes.c_int),
     "smoe_last_launch_count": ([], ctypes.c_int32),
@@ -179,6 +194,14 @@ def smoe_forward(cfg, x, T, w_router, bias, packed, out, ws=None, ws_bytes=None,
                                               _p(out), _p(ws), _ws_bytes(ws, ws_bytes), _s(stream)))
 
 
+def smoe_forward_diag(cfg, x, T, w_router, bias, packed, out, diag, ws=None, ws_bytes=None, stream=None):
+    """diag: a mapping with the smoe_diag_t fields (device tensors), e.g. from diag_buffers()."""
+    d = SmoeDiag(*[_p(diag[f]) for f in DIAG_FIELDS])
+    _check("smoe_forward_diag", lib().smoe_forward_diag(ctypes.byref(cfg), _p(x), T, _p(w_router), _p(bias),
+                                                        _p(packed), _p(out), ctypes.byref(d), _p(ws),
+                                                        _ws_bytes(ws, ws_bytes), _s(stream)))
+
+
 def smoe_get_device_error(ws, stream=None) -> int:
     code = ctypes.c_int32(0)
     _check("smoe_get_device_error", lib().smoe_get_device_error(_p(ws), ctypes.byref(code), _s(stream)))
@@ -219,6 +242,17 @@ def workspace(cfg: SmoeConfig, T: int, forward: bool = True, device="cuda"):
     import torch
     n = smoe_workspace_bytes(cfg, T) if forward else smoe_scratch_bytes(cfg, T)
     return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def diag_buffers(cfg: SmoeConfig, T: int, device="cuda") -> dict:
+    """Device arrays for smoe_forward_diag's outputs."""
+    import torch
+    E = cfg.n_experts
+    return {"expert_count": torch.empty(E, dtype=torch.int32, device=device),
+            "expert_norm_mean": torch.empty(E, dtype=torch.float32, device=device),
+            "expert_norm_max": torch.empty(E, dtype=torch.float32, device=device),
+            "token_confidence": torch.empty(max(T, 1), dtype=torch.float32, device=device),
+            "summary": torch.empty(SMOE_DIAG_SUMMARY, dtype=torch.float32, device=device)}
 
 
 def pack_weights(cfg, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, stream=None):

@@ -36,7 +36,7 @@ const char* const kNames[K_NUM_KERNELS] = {"router_logits", "router_topk",   "pe
                                            "permute_scan",  "permute_scatter", "gather_rows",
                                            "expert_gateup", "expert_down",   "combine",
                                            "pack_gateup",   "pack_down",     "router_split",
-                                           "router_gemm"};
+                                           "router_gemm",   "diag"};
 }  // namespace
 
 const char* kernel_name(int id) { return (id >= 0 && id < K_NUM_KERNELS) ? kNames[id] : "unknown"; }
@@ -90,6 +90,7 @@ WsLayout ws_layout(const smoe_config_t& c, int64_t T, int num_sms) {
     L.x_perm = o;    // only when smoe_forward materialises the permuted rows (large token tiles)
     if (choose_token_tile(c, T) > kGatherMaxTile) o += align_up((size_t)routed * H * 2);
     L.y = o;         o += align_up((size_t)(routed + T) * H * 2);
+    L.row_norm = o;  o += align_up((size_t)routed * 4);
     L.total = o;
     return L;
 }
@@ -288,12 +289,23 @@ smoe_status_t smoe_combine(const smoe_config_t* c, const smoe_bf16_t* y, const i
                                       static_cast<cudaStream_t>(stream)));
 }
 
-smoe_status_t smoe_forward(const smoe_config_t* c, const smoe_bf16_t* x, int64_t T, const float* w_router,
-                           const float* bias, const void* packed, smoe_bf16_t* out, void* ws, size_t ws_bytes,
-                           void* stream) {
+}  // extern "C"
+
+namespace {
+
+smoe_status_t forward_impl(const smoe_config_t* c, const smoe_bf16_t* x, int64_t T, const float* w_router,
+                           const float* bias, const void* packed, smoe_bf16_t* out, const smoe_diag_t* diag, void* ws,
+                           size_t ws_bytes, void* stream) {
     SMOE_TRY(smoe_check_config(c));
     SMOE_TRY(check_T(c, T));
     launches_reset();
+    if (diag != nullptr) {
+        SMOE_REQUIRE_PTR(diag->expert_count);
+        SMOE_REQUIRE_PTR(diag->expert_norm_mean);
+        SMOE_REQUIRE_PTR(diag->expert_norm_max);
+        SMOE_REQUIRE_PTR(diag->summary);
+        if (T > 0) SMOE_REQUIRE_PTR(diag->token_confidence);
+    }
     if (T == 0) return SMOE_OK;
     SMOE_REQUIRE_PTR(x);
     SMOE_REQUIRE_PTR(w_router);
@@ -311,8 +323,10 @@ smoe_status_t smoe_forward(const smoe_config_t* c, const smoe_bf16_t* x, int64_t
     int32_t* perm_row = at<int32_t>(ws, L.perm_row);
     int32_t* row_token = at<int32_t>(ws, L.row_token);
     uint16_t* y = at<uint16_t>(ws, L.y);
+    float* conf = diag != nullptr ? diag->token_confidence : nullptr;
+    float* row_norm = diag != nullptr ? at<float>(ws, L.row_norm) : nullptr;
     cudaError_t e = launch_route(*c, x, T, w_router, bias, idx, w, nullptr, at<float>(ws, L.route_partials), err,
-                                 sms, s);
+                                 sms, s, true, conf);
     // small token tiles: routed rows are gathered from x inside the expert GEMM (no permuted
     // copy); large tiles: one gather kernel writes x_perm and the GEMM loads whole tiles
     const bool gather = choose_token_tile(*c, T) <= kGatherMaxTile;
@@ -322,8 +336,28 @@ smoe_status_t smoe_forward(const smoe_config_t* c, const smoe_bf16_t* x, int64_t
                            x_perm, at<int32_t>(ws, L.perm_hist), at<int32_t>(ws, L.perm_base), err, s);
     if (e == cudaSuccess)
         e = launch_expert_ffn(*c, x, x_perm, row_token, offsets, T, packed, y, at<uint16_t>(ws, L.ffn_h), err, sms, s);
-    if (e == cudaSuccess) e = launch_combine(*c, y, perm_row, w, T, out, err, s);
+    if (e == cudaSuccess) e = launch_combine(*c, y, perm_row, w, T, out, err, s, row_norm);
+    if (e == cudaSuccess && diag != nullptr)
+        e = launch_diag(*c, T, row_norm, offsets, conf, diag->expert_count, diag->expert_norm_mean,
+                        diag->expert_norm_max, diag->summary, err, s);
     return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+smoe_status_t smoe_forward(const smoe_config_t* c, const smoe_bf16_t* x, int64_t T, const float* w_router,
+                           const float* bias, const void* packed, smoe_bf16_t* out, void* ws, size_t ws_bytes,
+                           void* stream) {
+    return forward_impl(c, x, T, w_router, bias, packed, out, nullptr, ws, ws_bytes, stream);
+}
+
+smoe_status_t smoe_forward_diag(const smoe_config_t* c, const smoe_bf16_t* x, int64_t T, const float* w_router,
+                                const float* bias, const void* packed, smoe_bf16_t* out, const smoe_diag_t* diag,
+                                void* ws, size_t ws_bytes, void* stream) {
+    if (diag == nullptr) return SMOE_ERR_INVALID_ARG;
+    return forward_impl(c, x, T, w_router, bias, packed, out, diag, ws, ws_bytes, stream);
 }
 
 smoe_status_t smoe_get_device_error(const void* ws, int32_t* code, void* stream) {

@@ -35,6 +35,7 @@ struct WsLayout {
     size_t ffn_h = 0;            // [T*k + T][I] bf16    (inside the union)
     size_t scratch_end = 0;
     size_t topk_idx = 0, topk_w = 0, counts = 0, offsets = 0, perm_row = 0, row_token = 0, x_perm = 0, y = 0;
+    size_t row_norm = 0;         // [T*k] fp32 (smoe_forward_diag)
     size_t total = 0;
 };
 WsLayout ws_layout(const smoe_config_t& c, int64_t T, int num_sms);
@@ -50,7 +51,7 @@ void launches_add(int n);
 enum KernelId {
     K_ROUTER_LOGITS = 0, K_ROUTER_TOPK, K_PERMUTE_HIST, K_PERMUTE_SCAN, K_PERMUTE_SCATTER, K_GATHER_ROWS,
     K_EXPERT_GATEUP, K_EXPERT_DOWN, K_COMBINE, K_PACK_GATEUP, K_PACK_DOWN, K_ROUTER_SPLIT, K_ROUTER_GEMM,
-    K_NUM_KERNELS
+    K_DIAG, K_NUM_KERNELS
 };
 const char* kernel_name(int id);
 
@@ -63,7 +64,7 @@ struct LaunchTimer {
 
 cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, const float* wr, const float* bias,
                          int32_t* topk_idx, float* topk_w, float* logits_opt, float* partials, int32_t* err,
-                         int num_sms, cudaStream_t s, bool allow_tc = true);
+                         int num_sms, cudaStream_t s, bool allow_tc = true, float* conf_opt = nullptr);
 
 cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* w_split, int e_pad, int E,
                                float* logits, int nt, int ksplit, int num_sms, cudaStream_t s);
@@ -88,8 +89,14 @@ cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const u
                               const int32_t* row_token, const int32_t* offsets, int64_t T, const void* packed,
                               uint16_t* y, uint16_t* h, int32_t* err, int num_sms, cudaStream_t s);
 
+// row_norm_opt: when set, also ||y[r]||_2 of every routed row r (fp32, [T*k]).
 cudaError_t launch_combine(const smoe_config_t& c, const uint16_t* y, const int32_t* perm_row, const float* topk_w,
-                           int64_t T, uint16_t* out, int32_t* err, cudaStream_t s);
+                           int64_t T, uint16_t* out, int32_t* err, cudaStream_t s, float* row_norm_opt = nullptr);
+
+// Per-expert output-norm statistics and the layer summary of smoe_forward_diag (one CTA).
+cudaError_t launch_diag(const smoe_config_t& c, int64_t T, const float* row_norm, const int32_t* offsets,
+                        const float* conf, int32_t* count, float* norm_mean, float* norm_max, float* summary,
+                        int32_t* err, cudaStream_t s);
 
 cudaError_t launch_pack(const smoe_config_t& c, const uint16_t* wg, const uint16_t* wu, const uint16_t* wd,
                         const uint16_t* sg, const uint16_t* su, const uint16_t* sd, void* packed, cudaStream_t s);

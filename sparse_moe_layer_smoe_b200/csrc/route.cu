@@ -162,7 +162,7 @@ template <int NPL>
 __global__ void __launch_bounds__(256)
 router_topk_kernel(const float* __restrict__ part, int splits, const float* __restrict__ bias, int T, int E, int k,
                    float scale, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-                   float* __restrict__ logits_out) {
+                   float* __restrict__ logits_out, float* __restrict__ conf_out) {
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
@@ -257,6 +257,7 @@ router_topk_kernel(const float* __restrict__ part, int splits, const float* __re
         topk_idx[(size_t)t * k + lane] = e_sel;
         topk_w[(size_t)t * k + lane] = scale * (s_sel / sum);
     }
+    if (conf_out != nullptr && lane == 0) conf_out[t] = sum / (float)k;   // routing confidence
 }
 
 // W_split[e][p*H + h] = piece p (0 = hi, 1 = mid, 2 = lo) of W_r[e][h]: hi = bf16(w),
@@ -317,12 +318,13 @@ cudaError_t launch_logits(const uint16_t* x, int64_t T, const float* wr, int E, 
 
 template <int NPL>
 cudaError_t launch_topk(const float* part, int splits, const float* bias, int64_t T, int E, int k, float scale,
-                        int32_t* idx, float* w, float* logits, cudaStream_t s) {
+                        int32_t* idx, float* w, float* logits, float* conf, cudaStream_t s) {
     const int warps = 8;
     {
         LaunchTimer lt(K_ROUTER_TOPK, s);
         router_topk_kernel<NPL><<<(unsigned)((T + warps - 1) / warps), warps * 32, 0, s>>>(part, splits, bias, (int)T,
-                                                                                           E, k, scale, idx, w, logits);
+                                                                                           E, k, scale, idx, w, logits,
+                                                                                           conf);
     }
     return cudaGetLastError();
 }
@@ -385,7 +387,7 @@ RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms, bool allo
 
 cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, const float* wr, const float* bias,
                          int32_t* topk_idx, float* topk_w, float* logits_opt, float* partials, int32_t* err,
-                         int num_sms, cudaStream_t s, bool allow_tc) {
+                         int num_sms, cudaStream_t s, bool allow_tc, float* conf_opt) {
     (void)err;
     const RouterPlan p = router_plan(c, T, num_sms, allow_tc);
     const int E = c.n_experts, H = c.hidden;
@@ -414,13 +416,13 @@ cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, c
     if (e != cudaSuccess) return e;
     const int npl = (E + 31) / 32;
     if (npl <= 4)
-        e = launch_topk<4>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, s);
+        e = launch_topk<4>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, s);
     else if (npl <= 9)
-        e = launch_topk<9>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, s);
+        e = launch_topk<9>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, s);
     else if (npl <= 16)
-        e = launch_topk<16>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, s);
+        e = launch_topk<16>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, s);
     else
-        e = launch_topk<32>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, s);
+        e = launch_topk<32>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, s);
     if (e == cudaSuccess) launches_add(n);
     return e;
 }

@@ -87,6 +87,26 @@ def test_argument_errors_before_any_launch():
     assert L.smoe_forward(ctypes.byref(bad), 16, 4, 16, 16, 16, 16, 256, 1 << 30, None) == smoe.SMOE_ERR_UNSUPPORTED
 
 
+def test_forward_diag_argument_errors():
+    L = smoe.lib()
+    c = smoe.config()
+    cp = ctypes.byref(c)
+    fneed = smoe.smoe_workspace_bytes(c, 64)
+    good = smoe.SmoeDiag(16, 16, 16, 16, 16)
+    # no diag struct, a missing array, a misaligned array: rejected before any launch
+    assert L.smoe_forward_diag(cp, 16, 64, 16, 16, 16, 16, None, 256, fneed, None) == smoe.SMOE_ERR_INVALID_ARG
+    for i, f in enumerate(smoe.DIAG_FIELDS):
+        for bad_ptr in (None, 24):
+            d = smoe.SmoeDiag(*[bad_ptr if j == i else 16 for j in range(len(smoe.DIAG_FIELDS))])
+            assert L.smoe_forward_diag(cp, 16, 64, 16, 16, 16, 16, ctypes.byref(d), 256, fneed,
+                                       None) == smoe.SMOE_ERR_INVALID_ARG, f
+    # the forward's own checks still apply (workspace too small), and T == 0 is a no-op
+    assert L.smoe_forward_diag(cp, 16, 64, 16, 16, 16, 16, ctypes.byref(good), 256, fneed - 1,
+                               None) == smoe.SMOE_ERR_WORKSPACE
+    z = smoe.SmoeDiag(16, 16, 16, None, 16)
+    assert L.smoe_forward_diag(cp, None, 0, None, None, None, None, ctypes.byref(z), None, 0, None) == 0
+
+
 def test_workspace_checks():
     L = smoe.lib()
     c = smoe.config()
