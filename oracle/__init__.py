@@ -5,10 +5,14 @@ leg may import this package. The CUDA library never imports it and shares no cod
 Parity status of each function (what pins it) is stated in ``tests/test_oracle_pins.py``.
 """
 from .diag import SUMMARY_FIELDS, Diagnostics, diagnostics, expert_output_norms, summarise
+from .fp8 import (E4M3_MAX, e4m3_code, e4m3_decode, e4m3_round, moe_sparse_fp8, quantize_rows, round_bf16,
+                  swiglu_ffn_fp8)
 from .moe import (NEAR_TIE_EPS, Route, bf16_to_f64, combine, f32_to_f64, moe_dense_masked, moe_given_selection,
                   moe_sparse, normalise, permute, route, router_logits, select_topk, sigmoid, silu, swiglu_ffn,
                   swiglu_hidden, valid_selections)
 
-__all__ = ["SUMMARY_FIELDS", "Diagnostics", "diagnostics", "expert_output_norms", "summarise", "NEAR_TIE_EPS",
+__all__ = ["SUMMARY_FIELDS", "Diagnostics", "diagnostics", "expert_output_norms", "summarise", "E4M3_MAX",
+           "e4m3_code", "e4m3_decode", "e4m3_round", "moe_sparse_fp8", "quantize_rows", "round_bf16",
+           "swiglu_ffn_fp8", "NEAR_TIE_EPS",
            "Route", "bf16_to_f64", "combine", "f32_to_f64", "moe_dense_masked", "moe_given_selection", "moe_sparse", "normalise", "permute", "route", "router_logits", "select_topk",
            "sigmoid", "silu", "swiglu_ffn", "swiglu_hidden", "valid_selections"]
