@@ -50,6 +50,7 @@ def parse_args(argv=None):
     p.add_argument("--cpu-sample-tokens", type=int, default=4)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--diag", action="store_true", help="time smoe_forward_diag (layer + monitoring outputs)")
+    p.add_argument("--fp8", action="store_true", help="time smoe_forward_fp8 (e4m3 experts, per-row scales)")
     return p.parse_args(argv)
 
 
@@ -272,17 +273,19 @@ def run_ours(args):
     x = synth.dev_x(w, device=dev)
     wr, bias = synth.dev_router(w, device=dev)
     experts = synth.dev_experts(w, device=dev)
-    packed = smoe.pack_weights(cfg, *experts)
+    packed = smoe.pack_weights_fp8(cfg, *experts) if args.fp8 else smoe.pack_weights(cfg, *experts)
     torch.cuda.synchronize()
     del experts
     torch.cuda.empty_cache()
-    ws = smoe.workspace(cfg, T, device=dev)
+    ws = smoe.workspace(cfg, T, device=dev, fp8=args.fp8)
     out = torch.empty(T, w.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
     diag = smoe.diag_buffers(cfg, T, device=dev) if args.diag else None
 
     def forward(x_):
-        if diag is None:
+        if args.fp8:
+            smoe.smoe_forward_fp8(cfg, x_, T, wr, bias, packed, out, ws)
+        elif diag is None:
             smoe.smoe_forward(cfg, x_, T, wr, bias, packed, out, ws)
         else:
             smoe.smoe_forward_diag(cfg, x_, T, wr, bias, packed, out, diag, ws)
@@ -347,8 +350,10 @@ def run_ours(args):
     peaks, peak_src = measured_peaks()
     dom = max(ktimes.items(), key=lambda kv: kv[1][1])[0] if ktimes else None
     H, I, E, k = w.H, w.I, w.E, w.k
-    gate_up_bytes = (touched + 1) * 2 * I * H * 2 + (T * k + T) * H * 2 + (T * k + T) * I * 2
-    down_bytes = (touched + 1) * H * I * 2 + (T * k + T) * I * 2 + (T * k + T) * H * 2
+    wb = 1 if args.fp8 else 2   # bytes per weight (e4m3 or bf16); e4m3 adds one fp32 scale per weight row
+    ab = 1 if args.fp8 else 2   # bytes per GEMM input activation
+    gate_up_bytes = (touched + 1) * 2 * I * (H * wb + (4 if args.fp8 else 0)) + (T * k + T) * H * ab + (T * k + T) * I * 2
+    down_bytes = (touched + 1) * H * (I * wb + (4 if args.fp8 else 0)) + (T * k + T) * I * ab + (T * k + T) * H * 2
     kern_bytes = {"expert_gateup": gate_up_bytes, "expert_down": down_bytes}
     kern_flops = {"expert_gateup": 2.0 * (T * k + T) * 2 * I * H, "expert_down": 2.0 * (T * k + T) * H * I}
     roof = None
@@ -356,27 +361,32 @@ def run_ours(args):
         launches, tot = ktimes[dom]
         avg_s = tot / launches / 1e3
         intensity = kern_flops[dom] / kern_bytes[dom]
-        ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        # the tensor peak of the contraction's own dtype: e4m3 = the measured bf16 peak x 2, the
+        # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+        tc_peak = peaks["bf16_tflops_sustained"] * (2.0 if args.fp8 else 1.0)
+        tc_src = ("MEASURED_PEAKS.json bf16_tflops_sustained x 2 (nominal e4m3 / bf16 ratio)" if args.fp8
+                  else "MEASURED_PEAKS.json bf16_tflops_sustained")
+        ridge = tc_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        traffic = profiled_traffic(dom, w.name + ("_fp8" if args.fp8 else ""))
         if intensity < ridge:
             ach = kern_bytes[dom] / avg_s / 1e9
             roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": ach / peaks["hbm_gbs"], "traffic": profiled_traffic(dom, w.name),
+                    "frac": ach / peaks["hbm_gbs"], "traffic": traffic,
                     "algorithmic_bytes": kern_bytes[dom], "avg_launch_ms": avg_s * 1e3,
                     "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_src})"}
         else:
             ach = kern_flops[dom] / avg_s / 1e12
-            roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
-                    "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"],
-                    "traffic": profiled_traffic(dom, w.name), "algorithmic_flops": kern_flops[dom],
-                    "avg_launch_ms": avg_s * 1e3,
-                    "peak_source": f"MEASURED_PEAKS.json bf16_tflops_sustained ({peak_src})"}
-    layer_bytes = (touched + 1) * 3 * H * I * 2 + E * H * 4 + 2 * T * H * 2
+            roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": tc_peak,
+                    "unit": "TFLOP/s", "frac": ach / tc_peak, "traffic": traffic, "algorithmic_flops": kern_flops[dom],
+                    "avg_launch_ms": avg_s * 1e3, "peak_source": f"{tc_src} ({peak_src})"}
+    layer_bytes = (touched + 1) * 3 * H * I * wb + E * H * 4 + 2 * T * H * 2
     layer_flops = 2.0 * T * (k + 1) * 3 * H * I
 
     line = {"metric": METRIC, "value": world * T / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {**workload_config(w), **({"diag": True} if args.diag else {})},
+            "vs_baseline": None, "dtype": "e4m3" if args.fp8 else "bf16", "data": "synthetic",
+            "config": {**workload_config(w), **({"diag": True} if args.diag else {}),
+                       **({"experts": "e4m3, per-row fp32 scales; router fp32"} if args.fp8 else {})},
             "layer": {"hbm_gbs": layer_bytes / (ms / 1e3) / 1e9, "tflops": layer_flops / (ms / 1e3) / 1e12,
                       "experts_touched": touched, "algorithmic_bytes": layer_bytes},
             "kernels_ms_per_step": {n: t / args.steps for n, (_, t) in sorted(ktimes.items(), key=lambda kv: -kv[1][1])},

@@ -214,6 +214,44 @@ SMOE_API smoe_status_t smoe_forward_diag(const smoe_config_t* cfg, const smoe_bf
                                 const float* w_router, const float* bias, const void* packed, smoe_bf16_t* out,
                                 const smoe_diag_t* diag, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- e4m3 (FP8) experts -------------------------------------------------------------------
+ * The Step 3.5 Flash summary (paperlayer.ai) fits the model into a 128 GB workstation budget,
+ * which calls for low-precision experts, but names no format. The format and quantiser here
+ * are readings, and the test oracle implements the same ones:
+ *   e4m3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, largest finite 448),
+ *   rounding to nearest even, finite values beyond +-448 saturating;
+ *   one fp32 scale per row of a matrix: s = max|row| / 448 (1 for an all-zero row), codes
+ *   e4m3(a / s) with a / s in IEEE fp32. Weight rows are output features (gate, up and down
+ *   rows of every expert); activation rows are tokens (x) or hidden rows (h).
+ * The expert: gate and up accumulate code products in fp32 on the tensor cores and are scaled
+ * by s_w * s_x; SiLU(gate) * up (with the SwiGLU clamp) is rounded to bf16 and quantised per
+ * row; the down product is scaled by s_w * s_h. Router, combine and shared add as in bf16.
+ * Packed layout (tile-major; every tile the GEMMs load is contiguous):
+ *   gate/up codes [(E+1)][I/128][H/128][256][128] (tile (g, mb, kb): the 128 gate rows of
+ *   features 128 mb .. +127, then the matching 128 up rows, K columns 128 kb .. +127),
+ *   down codes [(E+1)][H/128][I/128][128][128], then the fp32 scales: gate/up [(E+1)][2][I]
+ *   (gate rows, then up rows), down [(E+1)][H]. Each part starts on a 256-byte boundary. */
+
+/* Bytes of the packed e4m3 expert buffer smoe_pack_weights_fp8 writes. */
+SMOE_API smoe_status_t smoe_packed_weight_bytes_fp8(const smoe_config_t* cfg, size_t* bytes);
+
+/* Quantise and pack the experts (same inputs as smoe_pack_weights). Run once per layer. */
+SMOE_API smoe_status_t smoe_pack_weights_fp8(const smoe_config_t* cfg, const smoe_bf16_t* w_gate,
+                                const smoe_bf16_t* w_up, const smoe_bf16_t* w_down, const smoe_bf16_t* ws_gate,
+                                const smoe_bf16_t* ws_up, const smoe_bf16_t* ws_down, void* packed_fp8,
+                                void* stream);
+
+/* Workspace bytes of smoe_forward_fp8 for T tokens (smoe_forward's plus the e4m3 activations). */
+SMOE_API smoe_status_t smoe_workspace_bytes_fp8(const smoe_config_t* cfg, int64_t T, size_t* bytes);
+
+/* The whole layer with e4m3 experts: route (fp32, as smoe_forward) -> quantise x per token ->
+ * permute -> gate/up (e4m3 tensor cores) -> quantise h per row -> down -> combine. Arguments as
+ * smoe_forward, with packed_fp8 from smoe_pack_weights_fp8 and a workspace of at least
+ * smoe_workspace_bytes_fp8(cfg, T) bytes. */
+SMOE_API smoe_status_t smoe_forward_fp8(const smoe_config_t* cfg, const smoe_bf16_t* x, int64_t T,
+                                const float* w_router, const float* bias, const void* packed_fp8,
+                                smoe_bf16_t* out, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronise `stream` and read the workspace's device error word into *code
  * (SMOE_OK when no kernel recorded an error). */
 SMOE_API smoe_status_t smoe_get_device_error(const void* ws, int32_t* code, void* stream);
@@ -229,7 +267,8 @@ SMOE_API int32_t smoe_last_launch_count(void);
 typedef struct {
     char name[32];       /* kernel: router_logits, router_topk, permute_hist, permute_scan,
                             permute_scatter, gather_rows, expert_gateup, expert_down, combine,
-                            pack_gateup, pack_down, router_split, router_gemm, diag */
+                            pack_gateup, pack_down, router_split, router_gemm, diag,
+                            quantize_x, quantize_h, pack_fp8 */
     int32_t launches;    /* launches recorded */
     float total_ms;      /* summed event-to-event time of those launches */
 } smoe_kernel_time_t;

@@ -79,6 +79,10 @@ _SIGS = {
     "smoe_timing_end": ([ctypes.POINTER(SmoeKernelTime), ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)],
                         ctypes.c_int),
     "smoe_route_noalloc": ([_cfgp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "smoe_packed_weight_bytes_fp8": ([_cfgp, ctypes.POINTER(_sz)], ctypes.c_int),
+    "smoe_pack_weights_fp8": ([_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "smoe_workspace_bytes_fp8": ([_cfgp, _i64, ctypes.POINTER(_sz)], ctypes.c_int),
+    "smoe_forward_fp8": ([_cfgp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
 }
 
 _lib = None
@@ -202,6 +206,26 @@ def smoe_forward_diag(cfg, x, T, w_router, bias, packed, out, diag, ws=None, ws_
                                                         _ws_bytes(ws, ws_bytes), _s(stream)))
 
 
+def smoe_packed_weight_bytes_fp8(cfg: SmoeConfig) -> int:
+    return _bytes(lib().smoe_packed_weight_bytes_fp8, cfg)
+
+
+def smoe_workspace_bytes_fp8(cfg: SmoeConfig, T: int) -> int:
+    return _bytes(lib().smoe_workspace_bytes_fp8, cfg, T)
+
+
+def smoe_pack_weights_fp8(cfg, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, packed, stream=None) -> None:
+    _check("smoe_pack_weights_fp8", lib().smoe_pack_weights_fp8(ctypes.byref(cfg), _p(w_gate), _p(w_up), _p(w_down),
+                                                                 _p(ws_gate), _p(ws_up), _p(ws_down), _p(packed),
+                                                                 _s(stream)))
+
+
+def smoe_forward_fp8(cfg, x, T, w_router, bias, packed_fp8, out, ws=None, ws_bytes=None, stream=None):
+    _check("smoe_forward_fp8", lib().smoe_forward_fp8(ctypes.byref(cfg), _p(x), T, _p(w_router), _p(bias),
+                                                      _p(packed_fp8), _p(out), _p(ws), _ws_bytes(ws, ws_bytes),
+                                                      _s(stream)))
+
+
 def smoe_get_device_error(ws, stream=None) -> int:
     code = ctypes.c_int32(0)
     _check("smoe_get_device_error", lib().smoe_get_device_error(_p(ws), ctypes.byref(code), _s(stream)))
@@ -237,10 +261,14 @@ def _ws_bytes(ws, ws_bytes) -> int:
 
 
 # ------------------------------------------------------------------------------ conveniences (torch memory)
-def workspace(cfg: SmoeConfig, T: int, forward: bool = True, device="cuda"):
-    """A zeroed uint8 CUDA tensor large enough for smoe_forward (or the per-call entry points)."""
+def workspace(cfg: SmoeConfig, T: int, forward: bool = True, device="cuda", fp8: bool = False):
+    """A zeroed uint8 CUDA tensor large enough for smoe_forward (smoe_forward_fp8 with fp8=True,
+    or the per-call entry points with forward=False)."""
     import torch
-    n = smoe_workspace_bytes(cfg, T) if forward else smoe_scratch_bytes(cfg, T)
+    if fp8:
+        n = smoe_workspace_bytes_fp8(cfg, T)
+    else:
+        n = smoe_workspace_bytes(cfg, T) if forward else smoe_scratch_bytes(cfg, T)
     return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
 
 
@@ -259,6 +287,13 @@ def pack_weights(cfg, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, stream=None
     import torch
     packed = torch.empty(smoe_packed_weight_bytes(cfg), dtype=torch.uint8, device=w_gate.device)
     smoe_pack_weights(cfg, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, packed, stream)
+    return packed
+
+
+def pack_weights_fp8(cfg, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, stream=None):
+    import torch
+    packed = torch.empty(smoe_packed_weight_bytes_fp8(cfg), dtype=torch.uint8, device=w_gate.device)
+    smoe_pack_weights_fp8(cfg, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, packed, stream)
     return packed
 
 

@@ -36,7 +36,8 @@ const char* const kNames[K_NUM_KERNELS] = {"router_logits", "router_topk",   "pe
                                            "permute_scan",  "permute_scatter", "gather_rows",
                                            "expert_gateup", "expert_down",   "combine",
                                            "pack_gateup",   "pack_down",     "router_split",
-                                           "router_gemm",   "diag"};
+                                           "router_gemm",   "diag",        "quantize_x",
+                                           "quantize_h",    "pack_fp8"};
 }  // namespace
 
 const char* kernel_name(int id) { return (id >= 0 && id < K_NUM_KERNELS) ? kNames[id] : "unknown"; }
@@ -95,6 +96,20 @@ WsLayout ws_layout(const smoe_config_t& c, int64_t T, int num_sms) {
     return L;
 }
 
+// smoe_forward_fp8: the bf16 layout plus the e4m3 activations and their scales (the permuted
+// e4m3 rows, when needed, reuse the x_perm region).
+WsLayout ws_layout_fp8(const smoe_config_t& c, int64_t T, int num_sms) {
+    WsLayout L = ws_layout(c, T, num_sms);
+    const int64_t routed = T * c.top_k;
+    size_t o = L.total;
+    L.x_q = o;  o += align_up((size_t)T * c.hidden);
+    L.s_x = o;  o += align_up((size_t)T * 4);
+    L.h_q = o;  o += align_up((size_t)(routed + T) * c.inter);
+    L.s_h = o;  o += align_up((size_t)(routed + T) * 4);
+    L.total = o;
+    return L;
+}
+
 }  // namespace smoe
 
 using namespace smoe;
@@ -127,9 +142,10 @@ smoe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? SMOE_OK : S
         if ((p) != nullptr && !aligned16(p)) return SMOE_ERR_INVALID_ARG; \
     } while (0)
 
-smoe_status_t check_ws(const smoe_config_t* c, int64_t T, const void* ws, size_t ws_bytes, bool forward) {
+smoe_status_t check_ws(const smoe_config_t* c, int64_t T, const void* ws, size_t ws_bytes, bool forward,
+                       bool fp8 = false) {
     if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return SMOE_ERR_INVALID_ARG;
-    const WsLayout L = ws_layout(*c, T, num_sms_current_device());
+    const WsLayout L = fp8 ? ws_layout_fp8(*c, T, num_sms_current_device()) : ws_layout(*c, T, num_sms_current_device());
     if (ws_bytes < (forward ? L.total : L.scratch_end)) return SMOE_ERR_WORKSPACE;
     return SMOE_OK;
 }
@@ -184,6 +200,37 @@ smoe_status_t smoe_workspace_bytes(const smoe_config_t* c, int64_t T, size_t* by
     if (bytes == nullptr) return SMOE_ERR_INVALID_ARG;
     *bytes = ws_layout(*c, T, num_sms_current_device()).total;
     return SMOE_OK;
+}
+
+smoe_status_t smoe_workspace_bytes_fp8(const smoe_config_t* c, int64_t T, size_t* bytes) {
+    SMOE_TRY(smoe_check_config(c));
+    SMOE_TRY(check_T(c, T));
+    if (bytes == nullptr) return SMOE_ERR_INVALID_ARG;
+    *bytes = ws_layout_fp8(*c, T, num_sms_current_device()).total;
+    return SMOE_OK;
+}
+
+smoe_status_t smoe_packed_weight_bytes_fp8(const smoe_config_t* c, size_t* bytes) {
+    SMOE_TRY(smoe_check_config(c));
+    if (bytes == nullptr) return SMOE_ERR_INVALID_ARG;
+    *bytes = fp8_layout(*c).total;
+    return SMOE_OK;
+}
+
+smoe_status_t smoe_pack_weights_fp8(const smoe_config_t* c, const smoe_bf16_t* w_gate, const smoe_bf16_t* w_up,
+                                    const smoe_bf16_t* w_down, const smoe_bf16_t* ws_gate, const smoe_bf16_t* ws_up,
+                                    const smoe_bf16_t* ws_down, void* packed, void* stream) {
+    SMOE_TRY(smoe_check_config(c));
+    SMOE_REQUIRE_PTR(w_gate);
+    SMOE_REQUIRE_PTR(w_up);
+    SMOE_REQUIRE_PTR(w_down);
+    SMOE_REQUIRE_PTR(ws_gate);
+    SMOE_REQUIRE_PTR(ws_up);
+    SMOE_REQUIRE_PTR(ws_down);
+    SMOE_REQUIRE_PTR(packed);
+    launches_reset();
+    return cuda_status(launch_pack_fp8(*c, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, packed,
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 smoe_status_t smoe_packed_weight_bytes(const smoe_config_t* c, size_t* bytes) {
@@ -295,7 +342,7 @@ namespace {
 
 smoe_status_t forward_impl(const smoe_config_t* c, const smoe_bf16_t* x, int64_t T, const float* w_router,
                            const float* bias, const void* packed, smoe_bf16_t* out, const smoe_diag_t* diag, void* ws,
-                           size_t ws_bytes, void* stream) {
+                           size_t ws_bytes, void* stream, bool fp8 = false) {
     SMOE_TRY(smoe_check_config(c));
     SMOE_TRY(check_T(c, T));
     launches_reset();
@@ -312,9 +359,9 @@ smoe_status_t forward_impl(const smoe_config_t* c, const smoe_bf16_t* x, int64_t
     SMOE_REQUIRE_PTR(bias);
     SMOE_REQUIRE_PTR(packed);
     SMOE_REQUIRE_PTR(out);
-    SMOE_TRY(check_ws(c, T, ws, ws_bytes, true));
+    SMOE_TRY(check_ws(c, T, ws, ws_bytes, true, fp8));
     const int sms = num_sms_current_device();
-    const WsLayout L = ws_layout(*c, T, sms);
+    const WsLayout L = fp8 ? ws_layout_fp8(*c, T, sms) : ws_layout(*c, T, sms);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t* err = at<int32_t>(ws, L.err);
     int32_t* idx = at<int32_t>(ws, L.topk_idx);
@@ -331,11 +378,28 @@ smoe_status_t forward_impl(const smoe_config_t* c, const smoe_bf16_t* x, int64_t
     // copy); large tiles: one gather kernel writes x_perm and the GEMM loads whole tiles
     const bool gather = choose_token_tile(*c, T) <= kGatherMaxTile;
     uint16_t* x_perm = gather ? nullptr : at<uint16_t>(ws, L.x_perm);
-    if (e == cudaSuccess)
-        e = launch_permute(*c, idx, T, gather ? nullptr : x, at<int32_t>(ws, L.counts), offsets, perm_row, row_token,
-                           x_perm, at<int32_t>(ws, L.perm_hist), at<int32_t>(ws, L.perm_base), err, s);
-    if (e == cudaSuccess)
-        e = launch_expert_ffn(*c, x, x_perm, row_token, offsets, T, packed, y, at<uint16_t>(ws, L.ffn_h), err, sms, s);
+    if (!fp8) {
+        if (e == cudaSuccess)
+            e = launch_permute(*c, idx, T, gather ? nullptr : x, at<int32_t>(ws, L.counts), offsets, perm_row,
+                               row_token, x_perm, at<int32_t>(ws, L.perm_hist), at<int32_t>(ws, L.perm_base), err, s);
+        if (e == cudaSuccess)
+            e = launch_expert_ffn(*c, x, x_perm, row_token, offsets, T, packed, y, at<uint16_t>(ws, L.ffn_h), err, sms,
+                                  s);
+    } else {
+        // e4m3: x quantised per token; the permuted copy (large tiles) is of the e4m3 rows, moved
+        // by the same gather kernel as 2-byte pairs
+        uint8_t* x_q = at<uint8_t>(ws, L.x_q);
+        float* s_x = at<float>(ws, L.s_x);
+        if (e == cudaSuccess) e = launch_quantize_rows(x, T, c->hidden, x_q, s_x, K_QUANT_X, s);
+        if (e == cudaSuccess)
+            e = launch_permute(*c, idx, T, gather ? nullptr : reinterpret_cast<const uint16_t*>(x_q),
+                               at<int32_t>(ws, L.counts), offsets, perm_row, row_token, x_perm,
+                               at<int32_t>(ws, L.perm_hist), at<int32_t>(ws, L.perm_base), err, s, c->hidden / 2);
+        if (e == cudaSuccess)
+            e = launch_expert_ffn_fp8(*c, x_q, gather ? nullptr : reinterpret_cast<const uint8_t*>(x_perm), s_x,
+                                      row_token, offsets, T, packed, y, at<uint16_t>(ws, L.ffn_h),
+                                      at<uint8_t>(ws, L.h_q), at<float>(ws, L.s_h), err, sms, s);
+    }
     if (e == cudaSuccess) e = launch_combine(*c, y, perm_row, w, T, out, err, s, row_norm);
     if (e == cudaSuccess && diag != nullptr)
         e = launch_diag(*c, T, row_norm, offsets, conf, diag->expert_count, diag->expert_norm_mean,
@@ -351,6 +415,12 @@ smoe_status_t smoe_forward(const smoe_config_t* c, const smoe_bf16_t* x, int64_t
                            const float* bias, const void* packed, smoe_bf16_t* out, void* ws, size_t ws_bytes,
                            void* stream) {
     return forward_impl(c, x, T, w_router, bias, packed, out, nullptr, ws, ws_bytes, stream);
+}
+
+smoe_status_t smoe_forward_fp8(const smoe_config_t* c, const smoe_bf16_t* x, int64_t T, const float* w_router,
+                               const float* bias, const void* packed_fp8, smoe_bf16_t* out, void* ws, size_t ws_bytes,
+                               void* stream) {
+    return forward_impl(c, x, T, w_router, bias, packed_fp8, out, nullptr, ws, ws_bytes, stream, true);
 }
 
 smoe_status_t smoe_forward_diag(const smoe_config_t* c, const smoe_bf16_t* x, int64_t T, const float* w_router,

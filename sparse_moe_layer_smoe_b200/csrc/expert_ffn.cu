@@ -86,6 +86,11 @@ struct GemmParams {
     float* out_f32;           // [*, out_ld] fp32 (router)
     int32_t* err;
     int max_tiles;            // capacity of the token-tile table in shared memory
+    // e4m3 launches: acc * w_scale[feature] * act_scale[activation row's token or row]
+    const float* w_scale;     // gate/up: [E+1][2][n_out] (gate rows, then up rows); down: [E+1][n_out]
+    const float* act_scale;   // per token (gate/up) or per activation row (down)
+    const int32_t* scale_tok; // gate/up: routed activation row -> token (act_scale index); down: nullptr
+    int scale_shared_base;    // act_scale index of the shared group's first row (0, or T*k for down)
 };
 
 // What a launch computes: the down projection, the fused gate/up + SiLU*mul, or router logits.
@@ -143,14 +148,15 @@ __device__ __forceinline__ int tile_index(int nt) { return 31 - __clz(nt) - 4; }
 // N=240 MMAs; the columns past N are never stored.
 __device__ __forceinline__ int mma_cols(int nvalid, int nt) { return min(nt, (nvalid + 15) & ~15); }
 
-// Packed expert weights are tile-major: weight block bi (R rows), K columns 64 kb .. 64 kb + 63
-// form one contiguous R x 64 tile, viewed by the tensor map as rows of a [*][64] matrix.
-// Coordinates (x, y) of the BK-wide K slice kg of block bi (K = the reduction length).
-template <int BK>
+// Packed expert weights are tile-major: weight block bi (R rows) and K columns TK kb .. TK kb +
+// TK - 1 form one contiguous tile of R rows of 128 bytes (TK = 64 bf16 or 128 e4m3 elements),
+// viewed by the tensor map as rows of a [*][TK] matrix. Coordinates (x, y) of the EK-wide K
+// slice kg of block bi (K = the reduction length).
+template <int EK, int TK>
 __device__ __forceinline__ void weight_tile_xy(int bi, int kg, int K, int R, int& x, int& y) {
-    const int k0 = kg * BK;
-    x = k0 & 63;
-    y = (bi * (K / 64) + (k0 >> 6)) * R;
+    const int k0 = kg * EK;
+    x = k0 % TK;
+    y = (bi * (K / TK) + k0 / TK) * R;
 }
 
 // Work table. A token tile is (group g, tile nb) of nt rows; a unit is (tile, feature block
@@ -229,8 +235,12 @@ __device__ int build_tile_table(const int32_t* offsets, int E, int T, int routed
 // columns) into registers as packed bf16 pairs: SiLU(gate) * up for gate/up (after the SwiGLU
 // clamp when lim > 0), the plain value for down. 32-column TMEM loads, one wait each.
 // nch = number of 32-column chunks holding valid tokens.
-template <bool DUAL>
-__device__ __forceinline__ void epi_load(uint32_t t_row, int nt_max, int nch, float lim, uint32_t (&hv)[128]) {
+// With F8 (e4m3 operands) the accumulators are first scaled: by rs_g * s(col) (gate, or the down
+// output) and rs_u * s(col) (up), rs = this feature's weight-row scale and s(col) the activation
+// scale of the column, which lane j of the warp holds in cs[c] for column 32 c + j.
+template <bool DUAL, bool F8>
+__device__ __forceinline__ void epi_load(uint32_t t_row, int nt_max, int nch, float lim, uint32_t (&hv)[128],
+                                         float rs_g, float rs_u, const float (&cs)[8]) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         if (c < nch) {
@@ -242,8 +252,19 @@ __device__ __forceinline__ void epi_load(uint32_t t_row, int nt_max, int nch, fl
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 float v0 = __uint_as_float(a[2 * j]), v1 = __uint_as_float(a[2 * j + 1]);
+                float c0 = 1.f, c1 = 1.f;
+                if (F8) {
+                    c0 = __shfl_sync(0xFFFFFFFFu, cs[c], 2 * j);
+                    c1 = __shfl_sync(0xFFFFFFFFu, cs[c], 2 * j + 1);
+                    v0 *= rs_g * c0;
+                    v1 *= rs_g * c1;
+                }
                 if (DUAL) {
                     float u0 = __uint_as_float(b[2 * j]), u1 = __uint_as_float(b[2 * j + 1]);
+                    if (F8) {
+                        u0 *= rs_u * c0;
+                        u1 *= rs_u * c1;
+                    }
                     if (lim > 0.0f) {   // SwiGLU clamp: gate from above, up on both sides
                         v0 = fminf(v0, lim);
                         v1 = fminf(v1, lim);
@@ -275,7 +296,31 @@ __device__ __forceinline__ void epi_store(const uint32_t (&hv)[128], int nch, in
     }
 }
 
-template <int MODE, int BK>
+// e4m3 launches: lane j loads the activation scale of columns 32 c + j of a unit (0 past its
+// valid rows); issued before the accumulator wait, so the loads overlap the MMAs.
+__device__ __forceinline__ void load_col_scales(const GemmParams& p, const Unit& w, int nvalid, const int32_t* offs,
+                                                int lane, float (&cs)[8]) {
+    const int base = (w.g < p.E ? offs[w.g] : p.scale_shared_base) + w.nb * w.nt;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const int col = 32 * c + lane;
+        float v = 0.f;
+        if (col < nvalid) {
+            int idx = base + col;
+            if (p.scale_tok != nullptr && w.g < p.E) {
+                idx = p.scale_tok[idx];
+                if (idx < 0 || idx >= p.T) {   // corrupt token index: never read past the scales
+                    record_error(p.err, SMOE_ERR_DEVICE);
+                    idx = -1;
+                }
+            }
+            if (idx >= 0) v = p.act_scale[idx];
+        }
+        cs[c] = v;
+    }
+}
+
+template <int MODE, int BK, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     using C = GemmCfg<MODE, BK>;
@@ -300,7 +345,9 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
     const int MB = p.n_out / 128;
-    const int KB = p.K / BK / p.ksplit;   // k-blocks of one unit
+    constexpr int EK = F8 ? 128 : BK;     // K elements per stage (128-byte rows either way)
+    constexpr int TK = F8 ? 128 : 64;     // K elements per packed weight tile
+    const int KB = p.K / EK / p.ksplit;   // k-blocks of one unit
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -392,10 +439,10 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                         tma_load_2d(smem_u32(a_s), &maps.w, kg * BK, a_row, fb, pol_w);
                     } else {
                         int wx, wy;
-                        weight_tile_xy<BK>(w.g * MB + w.mb, kg, p.K, C::A_ROWS, wx, wy);
+                        weight_tile_xy<EK, TK>(w.g * MB + w.mb, kg, p.K, C::A_ROWS, wx, wy);
                         tma_load_2d(smem_u32(a_s), &maps.w, wx, wy, fb, pol_w);
                     }
-                    if (!gather) tma_load_2d(smem_u32(a_s + C::A_BYTES), bm, b_k * BK, b_row, fb, pol_a);
+                    if (!gather) tma_load_2d(smem_u32(a_s + C::A_BYTES), bm, b_k * EK, b_row, fb, pol_a);
                 }
                 __syncwarp(pmask);
                 if (gather) {
@@ -403,7 +450,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                     for (int j = 0; j < 2; ++j) {
                         const int c = lane + 32 * j;
                         if (c < nchunks)
-                            tma_gather4_2d(smem_u32(a_s + C::A_BYTES + c * 4 * BK * 2), bm, b_k * BK, tok[4 * j],
+                            tma_gather4_2d(smem_u32(a_s + C::A_BYTES + c * 4 * BK * 2), bm, b_k * EK, tok[4 * j],
                                            tok[4 * j + 1], tok[4 * j + 2], tok[4 * j + 3], fb, pol_a);
                     }
                 }
@@ -419,7 +466,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         __syncwarp(pmask);
     } else if (warp == 1 && lane == 0) {
         // ---------------------------------------------------------------- MMA issuer
-        const uint32_t idesc0 = idesc_bf16_f32(128, 0);
+        const uint32_t idesc0 = F8 ? idesc_e4m3_f32(128, 0) : idesc_bf16_f32(128, 0);
         int stage = 0, acc = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
@@ -441,10 +488,15 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 for (int kk = 0; kk < BK / 16; ++kk) {
                     const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
                     const uint64_t bdesc = smem_desc_kmajor<C::SW>(b_s + kk * 32);
-                    umma_f16_ss(d, smem_desc_kmajor<C::SW>(a_s + kk * 32), bdesc, idesc, accum);
-                    if (DUAL)
-                        umma_f16_ss(d + p.nt_max, smem_desc_kmajor<C::SW>(a_s + C::UP_OFFSET + kk * 32), bdesc, idesc,
-                                    accum);
+                    const uint64_t adesc = smem_desc_kmajor<C::SW>(a_s + kk * 32);
+                    if (F8) umma_f8_ss(d, adesc, bdesc, idesc, accum); else umma_f16_ss(d, adesc, bdesc, idesc, accum);
+                    if (DUAL) {
+                        const uint64_t udesc = smem_desc_kmajor<C::SW>(a_s + C::UP_OFFSET + kk * 32);
+                        if (F8)
+                            umma_f8_ss(d + p.nt_max, udesc, bdesc, idesc, accum);
+                        else
+                            umma_f16_ss(d + p.nt_max, udesc, bdesc, idesc, accum);
+                    }
                 }
                 umma_commit(smem_u32(&empty[stage]));
                 if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -476,6 +528,8 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             const int rows = group_rows(w.g, E, p.T, offs);
             const int out_base = (w.g < E ? offs[w.g] : p.shared_out_row) + w.nb * w.nt;
             const int nvalid = min(w.nt, rows - w.nb * w.nt);
+            float cs[8];
+            if (F8) load_col_scales(p, w, nvalid, offs, lane, cs);
             if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.err, abort_flag, true)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
@@ -496,7 +550,13 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             } else {
                 const int nch = (nvalid + 31) / 32;
                 uint32_t hv[128];
-                epi_load<DUAL>(t_row, p.nt_max, nch, w.g < E ? p.clamp_routed : p.clamp_shared, hv);
+                float rs_g = 1.f, rs_u = 1.f;
+                if (F8) {
+                    rs_g = p.w_scale[(size_t)(DUAL ? 2 * w.g : w.g) * p.n_out + f];
+                    if (DUAL) rs_u = p.w_scale[(size_t)(2 * w.g + 1) * p.n_out + f];
+                }
+                epi_load<DUAL, F8>(t_row, p.nt_max, nch, w.g < E ? p.clamp_routed : p.clamp_shared, hv, rs_g, rs_u,
+                                   cs);
                 tc_fence_before();
                 mbar_arrive(smem_u32(&tempty[acc]));   // accumulator free before the stores
                 epi_store(hv, nch, nvalid, p.out, dst0, p.out_ld);
@@ -535,7 +595,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
 // A cluster barrier before teardown keeps each CTA's shared memory and TMEM alive until the
 // pair's MMAs are done.
 // ------------------------------------------------------------------------------------------
-template <int MODE, int BK>
+template <int MODE, int BK, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     using C = GemmCfg<MODE, BK>;
@@ -563,7 +623,9 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
     const int E = p.E;
     const int MB = p.n_out / 128;       // 128-row blocks of a group's weights
     const int MBP = p.n_out / 256;      // 256-feature blocks handled by a pair
-    const int KB = p.K / BK;
+    constexpr int EK = F8 ? 128 : BK;     // K elements per stage (128-byte rows either way)
+    constexpr int TK = F8 ? 128 : 64;     // K elements per packed weight tile
+    const int KB = p.K / EK;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -628,9 +690,9 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
                 if (rank == 0) mbar_arrive_expect_tx(fb_local, tx);
                 uint8_t* a_s = tiles + (size_t)stage * STAGE_B;
                 int wx, wy;
-                weight_tile_xy<BK>(a_blk, kb, p.K, C::A_ROWS, wx, wy);
+                weight_tile_xy<EK, TK>(a_blk, kb, p.K, C::A_ROWS, wx, wy);
                 tma_load_2d_pair(smem_u32(a_s), &maps.w, wx, wy, fb_leader, pol_w);
-                tma_load_2d_pair(smem_u32(a_s + C::A_BYTES), bm, kb * BK, b_row, fb_leader, pol_a);
+                tma_load_2d_pair(smem_u32(a_s + C::A_BYTES), bm, kb * EK, b_row, fb_leader, pol_a);
                 armed |= 1u << stage;
                 armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                 if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -644,7 +706,7 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
         }
     } else if (warp == 1 && lane == 0 && rank == 0) {
         // ---------------------------------------------------------------- MMA issuer (first CTA)
-        const uint32_t idesc0 = idesc_bf16_f32(256, 0);
+        const uint32_t idesc0 = F8 ? idesc_e4m3_f32(256, 0) : idesc_bf16_f32(256, 0);
         int stage = 0, acc = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
@@ -666,10 +728,18 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
                 for (int kk = 0; kk < BK / 16; ++kk) {
                     const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
                     const uint64_t bdesc = smem_desc_kmajor<C::SW>(b_s + kk * 32);
-                    umma_f16_ss_pair(d, smem_desc_kmajor<C::SW>(a_s + kk * 32), bdesc, idesc, accum);
-                    if (DUAL)
-                        umma_f16_ss_pair(d + p.nt_max, smem_desc_kmajor<C::SW>(a_s + C::UP_OFFSET + kk * 32), bdesc,
-                                         idesc, accum);
+                    const uint64_t adesc = smem_desc_kmajor<C::SW>(a_s + kk * 32);
+                    if (F8)
+                        umma_f8_ss_pair(d, adesc, bdesc, idesc, accum);
+                    else
+                        umma_f16_ss_pair(d, adesc, bdesc, idesc, accum);
+                    if (DUAL) {
+                        const uint64_t udesc = smem_desc_kmajor<C::SW>(a_s + C::UP_OFFSET + kk * 32);
+                        if (F8)
+                            umma_f8_ss_pair(d + p.nt_max, udesc, bdesc, idesc, accum);
+                        else
+                            umma_f16_ss_pair(d + p.nt_max, udesc, bdesc, idesc, accum);
+                    }
                 }
                 const uint32_t eb = smem_u32(&empty[stage]);
                 umma_commit_pair(mapa_shared(eb, 0));
@@ -702,6 +772,8 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
             const int rows = group_rows(w.g, E, p.T, offs);
             const int out_base = (w.g < E ? offs[w.g] : p.shared_out_row) + w.nb * w.nt;
             const int nvalid = min(w.nt, rows - w.nb * w.nt);
+            float cs[8];
+            if (F8) load_col_scales(p, w, nvalid, offs, lane, cs);
             if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.err, abort_flag, true)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
@@ -709,7 +781,12 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
             const size_t dst0 = (size_t)out_base * p.out_ld + f;
             const int nch = (nvalid + 31) / 32;
             uint32_t hv[128];
-            epi_load<DUAL>(t_row, p.nt_max, nch, w.g < E ? p.clamp_routed : p.clamp_shared, hv);
+            float rs_g = 1.f, rs_u = 1.f;
+            if (F8) {
+                rs_g = p.w_scale[(size_t)(DUAL ? 2 * w.g : w.g) * p.n_out + f];
+                if (DUAL) rs_u = p.w_scale[(size_t)(2 * w.g + 1) * p.n_out + f];
+            }
+            epi_load<DUAL, F8>(t_row, p.nt_max, nch, w.g < E ? p.clamp_routed : p.clamp_shared, hv, rs_g, rs_u, cs);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));   // accumulator free
@@ -768,12 +845,32 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2D e4m3 tensor [rows][cols] (one byte per element) row-major; box = 128 columns (128 bytes,
+// swizzled) x box_rows.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A bf16 (bk-wide boxes) or, with u8, an e4m3 (128-wide boxes) activation map.
+bool make_any_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows, int bk, bool u8) {
+    return u8 ? make_map_u8(m, base, rows, cols, box_rows) : make_map(m, base, rows, cols, box_rows, bk);
+}
+
 // Activation maps for every token tile up to nt_max (larger entries repeat a valid map, unused).
-bool make_act_maps(CUtensorMap* maps, const void* base, uint64_t rows, uint64_t cols, int nt_max, int bk) {
+bool make_act_maps(CUtensorMap* maps, const void* base, uint64_t rows, uint64_t cols, int nt_max, int bk,
+                   bool u8 = false) {
     for (int i = 0; i < kNumTiles; ++i) {
         const int nt = 16 << i;
         if (nt <= nt_max) {
-            if (!make_map(&maps[i], base, rows, cols, nt, bk)) return false;
+            if (!make_any_map(&maps[i], base, rows, cols, nt, bk, u8)) return false;
         } else {
             maps[i] = maps[i - 1];
         }
@@ -794,7 +891,7 @@ int max_dynamic_smem() {
     return v;
 }
 
-template <int MODE>
+template <int MODE, bool F8 = false>
 cudaError_t run_gemm(const GemmMaps& maps, GemmParams p, int grid, cudaStream_t s) {
     constexpr int BK = SMOE_GEMM_BK;
     constexpr bool DUAL = MODE == MODE_GATEUP;
@@ -807,22 +904,23 @@ cudaError_t run_gemm(const GemmMaps& maps, GemmParams p, int grid, cudaStream_t 
     if (stages < 2) return cudaErrorInvalidConfiguration;
     p.stages = stages;
     const size_t smem = gemm_smem_bytes(stages, sb, p.E, p.max_tiles);
-    cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<MODE, BK, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     {
         LaunchTimer lt(MODE == MODE_GATEUP ? K_EXPERT_GATEUP : (MODE == MODE_DOWN ? K_EXPERT_DOWN : K_ROUTER_GEMM), s);
-        expert_gemm_kernel<MODE, BK><<<grid, kThreads, smem, s>>>(maps, p);
+        expert_gemm_kernel<MODE, BK, F8><<<grid, kThreads, smem, s>>>(maps, p);
     }
     return cudaGetLastError();
 }
 
 // Activation maps for CTA pairs: each CTA loads half of a token tile (box rows 8 << i).
-bool make_half_act_maps(CUtensorMap* maps, const void* base, uint64_t rows, uint64_t cols, int nt_max, int bk) {
+bool make_half_act_maps(CUtensorMap* maps, const void* base, uint64_t rows, uint64_t cols, int nt_max, int bk,
+                        bool u8 = false) {
     for (int i = 0; i < kNumTiles; ++i) {
         const int nt = 16 << i;
         if (nt <= nt_max) {
-            if (!make_map(&maps[i], base, rows, cols, nt / 2, bk)) return false;
+            if (!make_any_map(&maps[i], base, rows, cols, nt / 2, bk, u8)) return false;
         } else {
             maps[i] = maps[i - 1];
         }
@@ -830,7 +928,7 @@ bool make_half_act_maps(CUtensorMap* maps, const void* base, uint64_t rows, uint
     return true;
 }
 
-template <int MODE>
+template <int MODE, bool F8 = false>
 cudaError_t run_gemm_pair(const GemmMaps& maps, GemmParams p, int num_sms, cudaStream_t s) {
     constexpr int BK = SMOE_GEMM_BK;
     constexpr bool DUAL = MODE == MODE_GATEUP;
@@ -843,11 +941,12 @@ cudaError_t run_gemm_pair(const GemmMaps& maps, GemmParams p, int num_sms, cudaS
     if (stages < 2) return cudaErrorInvalidConfiguration;
     p.stages = stages;
     const size_t smem = gemm_smem_bytes(stages, sb, p.E, p.max_tiles);
-    auto kern = expert_gemm_pair_kernel<MODE, BK>;
+    auto kern = expert_gemm_pair_kernel<MODE, BK, F8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     // pairs resident at once (a GPC with an odd number of free SMs cannot host a pair there)
-    static int max_clusters[3] = {0, 0, 0};
+    static int max_clusters_by[2][3] = {{0, 0, 0}, {0, 0, 0}};
+    int* max_clusters = max_clusters_by[F8 ? 1 : 0];
     if (max_clusters[MODE] == 0) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(num_sms & ~1);
@@ -917,6 +1016,57 @@ cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const u
     GemmParams p2{offsets, E, (int)T, (int)routed, I, H, (int)routed, (int)routed, nt, 0, 0, H, H, nullptr, 0.f, 0.f, 1,
                   0, y, nullptr, err};
     e = pairs ? run_gemm_pair<MODE_DOWN>(m2, p2, num_sms, s) : run_gemm<MODE_DOWN>(m2, p2, num_sms, s);
+    if (e == cudaSuccess) launches_add(2);
+    return e;
+}
+
+cudaError_t launch_expert_ffn_fp8(const smoe_config_t& c, const uint8_t* x_q, const uint8_t* x_q_perm,
+                                  const float* s_x, const int32_t* row_token, const int32_t* offsets, int64_t T,
+                                  const void* packed_fp8, uint16_t* y, uint16_t* h, uint8_t* h_q, float* s_h,
+                                  int32_t* err, int num_sms, cudaStream_t s) {
+    constexpr int BK = SMOE_GEMM_BK;
+    const int E = c.n_experts, H = c.hidden, I = c.inter, k = c.top_k;
+    const int64_t routed = T * k;
+    const int nt = choose_token_tile(c, T);
+    const Fp8Layout L = fp8_layout(c);
+    const uint8_t* pk = static_cast<const uint8_t*>(packed_fp8);
+
+    GemmMaps m1, m2;
+    const bool gather = x_q_perm == nullptr;
+    const bool pairs = !gather && nt >= kPairMinTile && I % 256 == 0 && H % 256 == 0;
+    auto act_maps = [&](CUtensorMap* maps, const void* base, uint64_t rows, uint64_t cols) {
+        return pairs ? make_half_act_maps(maps, base, rows, cols, nt, BK, true)
+                     : make_act_maps(maps, base, rows, cols, nt, BK, true);
+    };
+    bool ok_act = gather ? make_map_u8(&m1.act[0], x_q, (uint64_t)T, H, 1) : act_maps(m1.act, x_q_perm, (uint64_t)routed, H);
+    if (gather)
+        for (int i = 1; i < kNumTiles; ++i) m1.act[i] = m1.act[0];
+    // packed codes, tile-major: viewed as [rows][128] with 256-row (gate/up) / 128-row (down) tiles
+    if (!ok_act || !make_map_u8(&m1.w, pk + L.gateup, (uint64_t)(E + 1) * 2 * I * (H / 128), 128, 256) ||
+        !act_maps(m1.sh, x_q, (uint64_t)T, H) ||
+        !make_map_u8(&m2.w, pk + L.down, (uint64_t)(E + 1) * H * (I / 128), 128, 128) ||
+        !act_maps(m2.act, h_q, (uint64_t)(routed + T), I))
+        return cudaErrorNotSupported;
+    for (int i = 0; i < kNumTiles; ++i) m2.sh[i] = m2.act[i];
+
+    GemmParams p1{offsets, E, (int)T, (int)routed, H, I, 0, (int)routed, nt, 0, 0, I, I, gather ? row_token : nullptr,
+                  c.swiglu_limit, c.swiglu_limit_shared, 1, 0, h, nullptr, err};
+    p1.w_scale = reinterpret_cast<const float*>(pk + L.gateup_scale);
+    p1.act_scale = s_x;
+    p1.scale_tok = row_token;
+    p1.scale_shared_base = 0;
+    cudaError_t e = pairs ? run_gemm_pair<MODE_GATEUP, true>(m1, p1, num_sms, s)
+                          : run_gemm<MODE_GATEUP, true>(m1, p1, num_sms, s);
+    if (e != cudaSuccess) return e;
+    e = launch_quantize_rows(h, routed + T, I, h_q, s_h, K_QUANT_H, s);
+    if (e != cudaSuccess) return e;
+    GemmParams p2{offsets, E, (int)T, (int)routed, I, H, (int)routed, (int)routed, nt, 0, 0, H, H, nullptr, 0.f, 0.f, 1,
+                  0, y, nullptr, err};
+    p2.w_scale = reinterpret_cast<const float*>(pk + L.down_scale);
+    p2.act_scale = s_h;
+    p2.scale_tok = nullptr;
+    p2.scale_shared_base = (int)routed;
+    e = pairs ? run_gemm_pair<MODE_DOWN, true>(m2, p2, num_sms, s) : run_gemm<MODE_DOWN, true>(m2, p2, num_sms, s);
     if (e == cudaSuccess) launches_add(2);
     return e;
 }

@@ -36,9 +36,11 @@ struct WsLayout {
     size_t scratch_end = 0;
     size_t topk_idx = 0, topk_w = 0, counts = 0, offsets = 0, perm_row = 0, row_token = 0, x_perm = 0, y = 0;
     size_t row_norm = 0;         // [T*k] fp32 (smoe_forward_diag)
+    size_t x_q = 0, s_x = 0, h_q = 0, s_h = 0;   // smoe_forward_fp8 only
     size_t total = 0;
 };
 WsLayout ws_layout(const smoe_config_t& c, int64_t T, int num_sms);
+WsLayout ws_layout_fp8(const smoe_config_t& c, int64_t T, int num_sms);
 
 int num_sms_current_device();
 
@@ -51,7 +53,7 @@ void launches_add(int n);
 enum KernelId {
     K_ROUTER_LOGITS = 0, K_ROUTER_TOPK, K_PERMUTE_HIST, K_PERMUTE_SCAN, K_PERMUTE_SCATTER, K_GATHER_ROWS,
     K_EXPERT_GATEUP, K_EXPERT_DOWN, K_COMBINE, K_PACK_GATEUP, K_PACK_DOWN, K_ROUTER_SPLIT, K_ROUTER_GEMM,
-    K_DIAG, K_NUM_KERNELS
+    K_DIAG, K_QUANT_X, K_QUANT_H, K_PACK_FP8, K_NUM_KERNELS
 };
 const char* kernel_name(int id);
 
@@ -71,7 +73,8 @@ cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16
 
 cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int64_t T, const uint16_t* x,
                            int32_t* counts, int32_t* offsets, int32_t* perm_row, int32_t* row_token,
-                           uint16_t* x_perm, int32_t* hist, int32_t* base, int32_t* err, cudaStream_t s);
+                           uint16_t* x_perm, int32_t* hist, int32_t* base, int32_t* err, cudaStream_t s,
+                           int gather_cols = 0);   // row width in 2-byte units for the x_perm gather (0: hidden)
 
 // Largest token tile of an expert-GEMM launch for T tokens (16..256).
 int choose_token_tile(const smoe_config_t& c, int64_t T);
@@ -103,5 +106,25 @@ cudaError_t launch_pack(const smoe_config_t& c, const uint16_t* wg, const uint16
 
 size_t packed_gateup_bytes(const smoe_config_t& c);
 size_t packed_down_bytes(const smoe_config_t& c);
+
+// ---- e4m3 experts (per-row scales; see smoe_pack_weights_fp8)
+struct Fp8Layout {
+    size_t gateup = 0, down = 0, gateup_scale = 0, down_scale = 0, total = 0;   // byte offsets, size
+};
+Fp8Layout fp8_layout(const smoe_config_t& c);
+
+cudaError_t launch_pack_fp8(const smoe_config_t& c, const uint16_t* wg, const uint16_t* wu, const uint16_t* wd,
+                            const uint16_t* sg, const uint16_t* su, const uint16_t* sd, void* packed, cudaStream_t s);
+
+// q[r][:] = e4m3(a[r][:] / s[r]), s[r] = max |a[r][:]| / 448 (1 for an all-zero row); one warp per row.
+cudaError_t launch_quantize_rows(const uint16_t* a, int64_t rows, int cols, uint8_t* q, float* scale, KernelId id,
+                                 cudaStream_t s);
+
+// Gate/up and down with e4m3 operands: x_q [T][H] (+ x_q_perm [T*k][H] or nullptr: gather mode),
+// s_x [T]; the SwiGLU hidden h (bf16) is quantised per row into h_q / s_h between the GEMMs.
+cudaError_t launch_expert_ffn_fp8(const smoe_config_t& c, const uint8_t* x_q, const uint8_t* x_q_perm,
+                                  const float* s_x, const int32_t* row_token, const int32_t* offsets, int64_t T,
+                                  const void* packed_fp8, uint16_t* y, uint16_t* h, uint8_t* h_q, float* s_h,
+                                  int32_t* err, int num_sms, cudaStream_t s);
 
 }  // namespace smoe

@@ -252,7 +252,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 
 cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int64_t T, const uint16_t* x,
                            int32_t* counts, int32_t* offsets, int32_t* perm_row, int32_t* row_token,
-                           uint16_t* x_perm, int32_t* hist, int32_t* base, int32_t* err, cudaStream_t s) {
+                           uint16_t* x_perm, int32_t* hist, int32_t* base, int32_t* err, cudaStream_t s,
+                           int gather_cols) {
     const int E = c.n_experts, k = c.top_k;
     const int nblk = (int)((T + TB - 1) / TB);
     cudaError_t e;
@@ -299,8 +300,8 @@ cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int6
         if (blocks > 148 * 32) blocks = 148 * 32;
         {
             LaunchTimer lt(K_GATHER_ROWS, s);
-            gather_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, row_token, offsets, E, (int)T, c.hidden, x_perm,
-                                                                err);
+            gather_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, row_token, offsets, E, (int)T,
+                                                                gather_cols > 0 ? gather_cols : c.hidden, x_perm, err);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         ++n;
