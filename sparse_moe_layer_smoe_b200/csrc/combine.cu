@@ -50,6 +50,8 @@ __global__ void __launch_bounds__(256, 3) combine_kernel(const uint16_t* __restr
     __shared__ float ws[kMaxK];
     __shared__ float red[NORMS ? 8 * 8 : 1];   // [warp][slot] partial sums of squares
     float sq[8];                               // NORMS, k <= 8: this thread's sums of squares per slot
+    pdl_wait();
+    pdl_launch_dependents();
 #pragma unroll
     for (int j = 0; j < 8; ++j) sq[j] = 0.f;
     const int t = blockIdx.x;
@@ -141,16 +143,16 @@ __global__ void __launch_bounds__(256, 3) combine_kernel(const uint16_t* __restr
 cudaError_t launch_combine(const smoe_config_t& c, const uint16_t* y, const int32_t* perm_row, const float* topk_w,
                            int64_t T, uint16_t* out, int32_t* err, cudaStream_t s, float* row_norm_opt) {
     const int threads = c.hidden / 8 >= 256 ? 256 : 128;
+    cudaError_t e;
     {
         LaunchTimer lt(K_COMBINE, s);
         if (row_norm_opt != nullptr)
-            combine_kernel<true><<<(unsigned)T, threads, 0, s>>>(y, perm_row, topk_w, (int)T, c.top_k, c.hidden, out,
-                                                                 err, row_norm_opt);
+            e = launch_pdl(combine_kernel<true>, dim3((unsigned)T), dim3(threads), 0, s, y, perm_row, topk_w, (int)T,
+                           c.top_k, c.hidden, out, err, row_norm_opt);
         else
-            combine_kernel<false><<<(unsigned)T, threads, 0, s>>>(y, perm_row, topk_w, (int)T, c.top_k, c.hidden, out,
-                                                                  err, nullptr);
+            e = launch_pdl(combine_kernel<false>, dim3((unsigned)T), dim3(threads), 0, s, y, perm_row, topk_w, (int)T,
+                           c.top_k, c.hidden, out, err, (float*)nullptr);
     }
-    cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) launches_add(1);
     return e;
 }

@@ -34,6 +34,14 @@ __device__ __forceinline__ uint8_t float_to_e4m3(float f) {
     return (uint8_t)__nv_cvt_float_to_fp8(f, __NV_SATFINITE, __NV_E4M3);
 }
 
+// Programmatic dependent launch. Every kernel of the layer starts with pdl_wait(): it returns
+// once the previous kernel in the stream has completed and its writes are visible (at once
+// when that kernel was not launched as a programmatic dependency). pdl_launch_dependents() then
+// lets the next kernel launch while this one runs, so its launch and placement overlap this
+// kernel's tail; that kernel waits in its own pdl_wait() before touching memory.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(kDiagThreads) diag_kernel(const float* __restr
     __shared__ float s_rank[4];   // means of rank (n-1)/2, n/2, 0 and n-1
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int routed = T * k;
+    pdl_wait();
+    pdl_launch_dependents();
     for (int i = tid; i <= E; i += kDiagThreads) s_off[i] = offsets[i];
     __syncthreads();
 
@@ -186,12 +188,12 @@ __global__ void __launch_bounds__(kDiagThreads) diag_kernel(const float* __restr
 cudaError_t launch_diag(const smoe_config_t& c, int64_t T, const float* row_norm, const int32_t* offsets,
                         const float* conf, int32_t* count, float* norm_mean, float* norm_max, float* summary,
                         int32_t* err, cudaStream_t s) {
+    cudaError_t e;
     {
         LaunchTimer lt(K_DIAG, s);
-        diag_kernel<<<1, kDiagThreads, 0, s>>>(row_norm, offsets, conf, c.n_experts, (int)T, c.top_k, count,
-                                               norm_mean, norm_max, summary, err);
+        e = launch_pdl(diag_kernel, dim3(1), dim3(kDiagThreads), 0, s, row_norm, offsets, conf, c.n_experts, (int)T,
+                       c.top_k, count, norm_mean, norm_max, summary, err);
     }
-    cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) launches_add(1);
     return e;
 }

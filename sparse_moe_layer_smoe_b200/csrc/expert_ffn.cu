@@ -342,6 +342,8 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     int32_t* ttab = reinterpret_cast<int32_t*>(tmem_slot + 4);     // token tiles [max_tiles]
     int32_t* offs = ttab + p.max_tiles;                              // [E+1]
 
+    pdl_wait();
+    pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
     const int MB = p.n_out / 128;
@@ -617,6 +619,8 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
     int32_t* ttab = reinterpret_cast<int32_t*>(tmem_slot + 4);     // token tiles [max_tiles]
     int32_t* offs = ttab + p.max_tiles;                              // [E+1]
 
+    pdl_wait();
+    pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
@@ -909,9 +913,8 @@ cudaError_t run_gemm(const GemmMaps& maps, GemmParams p, int grid, cudaStream_t 
     if (e != cudaSuccess) return e;
     {
         LaunchTimer lt(MODE == MODE_GATEUP ? K_EXPERT_GATEUP : (MODE == MODE_DOWN ? K_EXPERT_DOWN : K_ROUTER_GEMM), s);
-        expert_gemm_kernel<MODE, BK, F8><<<grid, kThreads, smem, s>>>(maps, p);
+        return launch_pdl(expert_gemm_kernel<MODE, BK, F8>, dim3(grid), dim3(kThreads), smem, s, maps, p);
     }
-    return cudaGetLastError();
 }
 
 // Activation maps for CTA pairs: each CTA loads half of a token tile (box rows 8 << i).
@@ -960,9 +963,8 @@ cudaError_t run_gemm_pair(const GemmMaps& maps, GemmParams p, int num_sms, cudaS
     const int pairs = std::min(num_sms / 2, max_clusters[MODE]);
     {
         LaunchTimer lt(MODE == MODE_GATEUP ? K_EXPERT_GATEUP : K_EXPERT_DOWN, s);
-        kern<<<2 * pairs, kThreads, smem, s>>>(maps, p);
+        return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), smem, s, maps, p);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace

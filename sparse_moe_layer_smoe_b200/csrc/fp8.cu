@@ -65,6 +65,8 @@ __device__ __forceinline__ float quantize_row_warp(const uint16_t* __restrict__ 
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const uint16_t* __restrict__ a, int64_t rows, int cols,
                                                             uint8_t* __restrict__ q, float* __restrict__ scale) {
     const int lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_launch_dependents();
     for (int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += (int64_t)gridDim.x * 8) {
         uint2* dst = reinterpret_cast<uint2*>(q + (size_t)r * cols);
         const float sc = quantize_row_warp(a + (size_t)r * cols, cols, [&](int v, uint2 c) { dst[v] = c; });
@@ -148,11 +150,11 @@ cudaError_t launch_quantize_rows(const uint16_t* a, int64_t rows, int cols, uint
     int64_t blocks = (rows + 7) / 8;
     if (blocks > 148 * 16) blocks = 148 * 16;
     if (blocks < 1) blocks = 1;
+    cudaError_t e;
     {
         LaunchTimer lt(id, s);
-        quantize_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(a, rows, cols, q, scale);
+        e = launch_pdl(quantize_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s, a, rows, cols, q, scale);
     }
-    cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) launches_add(1);
     return e;
 }

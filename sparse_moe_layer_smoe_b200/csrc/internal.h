@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/stepmoe.h"
 
 namespace smoe {
@@ -63,6 +65,26 @@ struct LaunchTimer {
     LaunchTimer(KernelId id, cudaStream_t s);
     ~LaunchTimer();   // records the end event after the launch statement(s) in scope
 };
+
+#ifndef SMOE_PDL
+#define SMOE_PDL 1   // launch the layer's kernels as programmatic dependents (0: plain stream order)
+#endif
+
+// Launch as a programmatic dependent of the previous kernel in the stream (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = SMOE_PDL ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, const float* wr, const float* bias,
                          int32_t* topk_idx, float* topk_w, float* logits_opt, float* partials, int32_t* err,

@@ -44,6 +44,8 @@ __device__ __forceinline__ bool entry_valid(const int32_t* idx, int t, int j, in
 
 __global__ void __launch_bounds__(TB) permute_hist_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
                                                           int32_t* __restrict__ hist, int32_t* err) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ int32_t sh[];
     for (int e = threadIdx.x; e < E; e += TB) sh[e] = 0;
     __syncthreads();
@@ -60,6 +62,8 @@ __global__ void __launch_bounds__(TB) permute_hist_kernel(const int32_t* __restr
 __global__ void __launch_bounds__(1024) permute_scan_kernel(const int32_t* __restrict__ hist, int nblk, int E,
                                                             int32_t* __restrict__ base, int32_t* __restrict__ counts,
                                                             int32_t* __restrict__ offsets) {
+    pdl_wait();
+    pdl_launch_dependents();
     __shared__ int32_t warp_tot[32];
     const int e = threadIdx.x;
     int32_t run = 0;
@@ -100,6 +104,8 @@ __global__ void __launch_bounds__(TB) permute_scatter_kernel(const int32_t* __re
                                                              const int32_t* __restrict__ offsets,
                                                              int32_t* __restrict__ perm_row,
                                                              int32_t* __restrict__ row_token, int32_t* err) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ uint32_t smem[];
     uint32_t* wmask = smem;                                        // [WARPS][E]
     int32_t* wbase = reinterpret_cast<int32_t*>(smem + WARPS * E);  // [WARPS][E]
@@ -153,6 +159,8 @@ __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(const int3
                                                                       int32_t* __restrict__ offsets,
                                                                       int32_t* __restrict__ perm_row,
                                                                       int32_t* __restrict__ row_token, int32_t* err) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ uint32_t smem[];
     uint32_t* wmask = smem;                                                  // [warps][E]
     int32_t* wbase = reinterpret_cast<int32_t*>(smem + kSmallWarps * E);     // [warps][E]
@@ -225,6 +233,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
                                                           const int32_t* __restrict__ row_token,
                                                           const int32_t* __restrict__ offsets, int E, int T, int H,
                                                           uint16_t* __restrict__ x_perm, int32_t* err) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int nrows = offsets[E];
     const int lane = threadIdx.x & 31;
     const int vec = H / 8;
@@ -266,23 +276,24 @@ cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int6
         }
         {
             LaunchTimer lt(K_PERMUTE_SCATTER, s);
-            permute_small_kernel<<<1, kSmallThreads, small_sm, s>>>(topk_idx, (int)T, k, E, counts, offsets, perm_row,
-                                                                    row_token, err);
+            e = launch_pdl(permute_small_kernel, dim3(1), dim3(kSmallThreads), small_sm, s, topk_idx, (int)T, k, E,
+                           counts, offsets, perm_row, row_token, err);
         }
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (e != cudaSuccess) return e;
         n = 1;
     } else {
         {
             LaunchTimer lt(K_PERMUTE_HIST, s);
-            permute_hist_kernel<<<nblk, TB, E * sizeof(int32_t), s>>>(topk_idx, (int)T, k, E, hist, err);
+            e = launch_pdl(permute_hist_kernel, dim3(nblk), dim3(TB), E * sizeof(int32_t), s, topk_idx, (int)T, k, E,
+                           hist, err);
         }
-        e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         {
             LaunchTimer lt(K_PERMUTE_SCAN, s);
-            permute_scan_kernel<<<1, 1024, 0, s>>>(hist, nblk, E, base, counts, offsets);
+            e = launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, s, (const int32_t*)hist, nblk, E, base, counts,
+                           offsets);
         }
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (e != cudaSuccess) return e;
         const size_t sm = 2 * WARPS * E * sizeof(uint32_t);
         if (sm > 48 * 1024) {
             e = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
@@ -290,9 +301,10 @@ cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int6
         }
         {
             LaunchTimer lt(K_PERMUTE_SCATTER, s);
-            permute_scatter_kernel<<<nblk, TB, sm, s>>>(topk_idx, (int)T, k, E, base, offsets, perm_row, row_token, err);
+            e = launch_pdl(permute_scatter_kernel, dim3(nblk), dim3(TB), sm, s, topk_idx, (int)T, k, E,
+                           (const int32_t*)base, (const int32_t*)offsets, perm_row, row_token, err);
         }
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (e != cudaSuccess) return e;
     }
     if (x != nullptr && x_perm != nullptr) {
         const int64_t rows = T * k;
@@ -300,10 +312,10 @@ cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int6
         if (blocks > 148 * 32) blocks = 148 * 32;
         {
             LaunchTimer lt(K_GATHER_ROWS, s);
-            gather_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, row_token, offsets, E, (int)T,
-                                                                gather_cols > 0 ? gather_cols : c.hidden, x_perm, err);
+            e = launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s, x, (const int32_t*)row_token,
+                           (const int32_t*)offsets, E, (int)T, gather_cols > 0 ? gather_cols : c.hidden, x_perm, err);
         }
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (e != cudaSuccess) return e;
         ++n;
     }
     launches_add(n);

@@ -45,6 +45,8 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ w
                      int T, int E, int H, int k_len) {
     using P = RouterTile<TM, TE, RM, RE, KC_>;
     constexpr int KC = P::KC;
+    pdl_wait();
+    pdl_launch_dependents();
     // two stages of x [KC][TM+1] and W_r [KC][TE+1]; +1 padding: the transposing stores below
     // hit 32 distinct banks
     extern __shared__ float rsm[];
@@ -163,6 +165,8 @@ __global__ void __launch_bounds__(256)
 router_topk_kernel(const float* __restrict__ part, int splits, const float* __restrict__ bias, int T, int E, int k,
                    float scale, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                    float* __restrict__ logits_out, float* __restrict__ conf_out) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
@@ -267,6 +271,8 @@ router_topk_kernel(const float* __restrict__ part, int splits, const float* __re
 // Grid: (H/4/256 rounded up, e_pad); thread = 4 consecutive elements of row blockIdx.y.
 __global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ wr, int E, int H,
                                                            uint16_t* __restrict__ w_split) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int e = blockIdx.y;
     const int c = blockIdx.x * 256 + threadIdx.x;   // 4-element column group
     if (4 * c >= H) return;
@@ -311,9 +317,9 @@ cudaError_t launch_logits(const uint16_t* x, int64_t T, const float* wr, int E, 
     }
     {
         LaunchTimer lt(K_ROUTER_LOGITS, s);
-        router_logits_kernel<TM, TE, RM, RE, KC><<<grid, P::THREADS, smem, s>>>(x, wr, part, (int)T, E, H, H / splits);
+        return launch_pdl(router_logits_kernel<TM, TE, RM, RE, KC>, grid, dim3(P::THREADS), smem, s, x, wr, part,
+                          (int)T, E, H, H / splits);
     }
-    return cudaGetLastError();
 }
 
 template <int NPL>
@@ -322,11 +328,9 @@ cudaError_t launch_topk(const float* part, int splits, const float* bias, int64_
     const int warps = 8;
     {
         LaunchTimer lt(K_ROUTER_TOPK, s);
-        router_topk_kernel<NPL><<<(unsigned)((T + warps - 1) / warps), warps * 32, 0, s>>>(part, splits, bias, (int)T,
-                                                                                           E, k, scale, idx, w, logits,
-                                                                                           conf);
+        return launch_pdl(router_topk_kernel<NPL>, dim3((unsigned)((T + warps - 1) / warps)), dim3(warps * 32), 0, s,
+                          part, splits, bias, (int)T, E, k, scale, idx, w, logits, conf);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace
@@ -398,10 +402,10 @@ cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, c
         uint16_t* w_split = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(partials) + logit_b);
         {
             LaunchTimer lt(K_ROUTER_SPLIT, s);
-            router_split_kernel<<<dim3((unsigned)((H / 4 + 255) / 256), (unsigned)p.e_pad), 256, 0, s>>>(wr, E, H,
-                                                                                                       w_split);
+            e = launch_pdl(router_split_kernel, dim3((unsigned)((H / 4 + 255) / 256), (unsigned)p.e_pad), dim3(256), 0,
+                           s, wr, E, H, w_split);
         }
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (e != cudaSuccess) return e;
         e = launch_router_gemm(x, T, H, w_split, p.e_pad, E, partials, p.nt, p.splits, num_sms, s);
         n = 3;
     } else if (p.wide) {
