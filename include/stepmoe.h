@@ -259,6 +259,15 @@ SMOE_API smoe_status_t smoe_get_device_error(const void* ws, int32_t* code, void
 /* Reset the device error word to SMOE_OK (asynchronous on `stream`). */
 SMOE_API smoe_status_t smoe_clear_device_error(void* ws, void* stream);
 
+/* Failure-detection self-test: one thread waits, through the bounded mbarrier wait every GEMM
+ * role uses, on a barrier nothing arrives at, with the given limit (1 ns .. 1 s). The wait gives
+ * up after limit_ns, records SMOE_ERR_TIMEOUT in the workspace's error word (read it with
+ * smoe_get_device_error) and the kernel exits normally, leaving the context usable. If
+ * elapsed_ns_opt (device, 8-byte aligned) is set, the measured wait is written there. Needs only
+ * the workspace's first 256 bytes. Returns SMOE_ERR_INVALID_ARG for a limit outside the range or
+ * a misaligned pointer. (A library operation of its own; the pages have no counterpart.) */
+SMOE_API smoe_status_t smoe_selftest_wait_timeout(uint64_t limit_ns, uint64_t* elapsed_ns_opt, void* ws, void* stream);
+
 /* Number of kernel launches the last successful call on this host thread enqueued. */
 SMOE_API int32_t smoe_last_launch_count(void);
 

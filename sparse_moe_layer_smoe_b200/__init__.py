@@ -83,6 +83,7 @@ _SIGS = {
     "smoe_pack_weights_fp8": ([_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "smoe_workspace_bytes_fp8": ([_cfgp, _i64, ctypes.POINTER(_sz)], ctypes.c_int),
     "smoe_forward_fp8": ([_cfgp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "smoe_selftest_wait_timeout": ([ctypes.c_uint64, _vp, _vp, _vp], ctypes.c_int),
 }
 
 _lib = None
@@ -224,6 +225,11 @@ def smoe_forward_fp8(cfg, x, T, w_router, bias, packed_fp8, out, ws=None, ws_byt
     _check("smoe_forward_fp8", lib().smoe_forward_fp8(ctypes.byref(cfg), _p(x), T, _p(w_router), _p(bias),
                                                       _p(packed_fp8), _p(out), _p(ws), _ws_bytes(ws, ws_bytes),
                                                       _s(stream)))
+
+
+def smoe_selftest_wait_timeout(limit_ns, elapsed_ns=None, ws=None, stream=None) -> None:
+    _check("smoe_selftest_wait_timeout", lib().smoe_selftest_wait_timeout(int(limit_ns), _p(elapsed_ns), _p(ws),
+                                                                          _s(stream)))
 
 
 def smoe_get_device_error(ws, stream=None) -> int:

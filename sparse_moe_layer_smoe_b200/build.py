@@ -5,7 +5,7 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libstepmoe.so")
-SOURCES = ["api.cu", "route.cu", "permute.cu", "expert_ffn.cu", "combine.cu", "pack.cu", "noalloc.cu", "diag.cu", "fp8.cu"]
+SOURCES = ["api.cu", "route.cu", "permute.cu", "expert_ffn.cu", "combine.cu", "pack.cu", "noalloc.cu", "diag.cu", "fp8.cu", "selftest.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17", "-shared",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]
 

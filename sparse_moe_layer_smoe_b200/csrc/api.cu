@@ -430,6 +430,16 @@ smoe_status_t smoe_forward_diag(const smoe_config_t* c, const smoe_bf16_t* x, in
     return forward_impl(c, x, T, w_router, bias, packed, out, diag, ws, ws_bytes, stream);
 }
 
+smoe_status_t smoe_selftest_wait_timeout(uint64_t limit_ns, uint64_t* elapsed_ns_opt, void* ws, void* stream) {
+    if (limit_ns == 0 || limit_ns > 1000000000ull) return SMOE_ERR_INVALID_ARG;
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return SMOE_ERR_INVALID_ARG;
+    if (elapsed_ns_opt != nullptr && (reinterpret_cast<uintptr_t>(elapsed_ns_opt) & 7u) != 0)
+        return SMOE_ERR_INVALID_ARG;
+    launches_reset();
+    return cuda_status(launch_wait_selftest(static_cast<int32_t*>(ws), limit_ns, elapsed_ns_opt,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 smoe_status_t smoe_get_device_error(const void* ws, int32_t* code, void* stream) {
     if (ws == nullptr || code == nullptr) return SMOE_ERR_INVALID_ARG;
     int32_t v = 0;

@@ -87,21 +87,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // SMOE_ERR_TIMEOUT and raising *abort) when the time limit passes. With check_abort, it also
 // returns false as soon as another role of the CTA has raised *abort; drain waits (loads or
 // MMAs still in flight before the CTA exits) pass check_abort = false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* err, volatile int* abort,
-                                          bool check_abort) {
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, int32_t* err, volatile int* abort,
+                                              bool check_abort, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 255u) == 0) {
             if (check_abort && *abort) return false;
-            if (globaltimer_ns() - t0 > SMOE_WAIT_LIMIT_NS) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 record_error(err, SMOE_ERR_TIMEOUT);
                 *abort = 1;
                 return false;
             }
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* err, volatile int* abort,
+                                          bool check_abort) {
+    return mbar_wait_for(bar, parity, err, abort, check_abort, SMOE_WAIT_LIMIT_NS);
 }
 
 // ---------------------------------------------------------------------------------------------

@@ -126,6 +126,9 @@ cudaError_t launch_diag(const smoe_config_t& c, int64_t T, const float* row_norm
 cudaError_t launch_pack(const smoe_config_t& c, const uint16_t* wg, const uint16_t* wu, const uint16_t* wd,
                         const uint16_t* sg, const uint16_t* su, const uint16_t* sd, void* packed, cudaStream_t s);
 
+// The bounded-wait self-test (smoe_selftest_wait_timeout).
+cudaError_t launch_wait_selftest(int32_t* err, uint64_t limit_ns, uint64_t* elapsed_ns, cudaStream_t s);
+
 size_t packed_gateup_bytes(const smoe_config_t& c);
 size_t packed_down_bytes(const smoe_config_t& c);
 

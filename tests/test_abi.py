@@ -107,6 +107,36 @@ def test_forward_diag_argument_errors():
     assert L.smoe_forward_diag(cp, None, 0, None, None, None, None, ctypes.byref(z), None, 0, None) == 0
 
 
+def test_fp8_entry_points_argument_errors_and_sizes():
+    L = smoe.lib()
+    c = smoe.config()
+    cp = ctypes.byref(c)
+    # packed e4m3 size: one byte per weight + one fp32 scale per weight row, each part 256-aligned
+    E1, H, I = 289, 4096, 1280
+    al = lambda n: (n + 255) // 256 * 256
+    assert smoe.smoe_packed_weight_bytes_fp8(c) == al(E1 * 2 * I * H) + al(E1 * H * I) + al(E1 * 2 * I * 4) + al(E1 * H * 4)
+    assert smoe.smoe_workspace_bytes_fp8(c, 64) > smoe.smoe_workspace_bytes(c, 64)
+    assert L.smoe_pack_weights_fp8(cp, 16, 16, 16, 16, 16, None, 16, None) == smoe.SMOE_ERR_INVALID_ARG
+    assert L.smoe_pack_weights_fp8(cp, 16, 16, 16, 16, 16, 16, 24, None) == smoe.SMOE_ERR_INVALID_ARG
+    need = smoe.smoe_workspace_bytes_fp8(c, 64)
+    assert L.smoe_forward_fp8(cp, 16, 64, 16, 16, None, 16, 256, need, None) == smoe.SMOE_ERR_INVALID_ARG
+    # the bf16 forward's workspace is too small for the e4m3 forward
+    assert L.smoe_forward_fp8(cp, 16, 64, 16, 16, 16, 16, 256, smoe.smoe_workspace_bytes(c, 64),
+                              None) == smoe.SMOE_ERR_WORKSPACE
+    assert L.smoe_forward_fp8(cp, None, 0, None, None, None, None, None, 0, None) == 0
+    bad = smoe.config(inter=192)
+    assert L.smoe_forward_fp8(ctypes.byref(bad), 16, 4, 16, 16, 16, 16, 256, 1 << 30, None) == smoe.SMOE_ERR_UNSUPPORTED
+
+
+def test_selftest_argument_checks():
+    L = smoe.lib()
+    assert L.smoe_selftest_wait_timeout(0, None, 256, None) == smoe.SMOE_ERR_INVALID_ARG
+    assert L.smoe_selftest_wait_timeout(2_000_000_000, None, 256, None) == smoe.SMOE_ERR_INVALID_ARG
+    assert L.smoe_selftest_wait_timeout(1000, None, None, None) == smoe.SMOE_ERR_INVALID_ARG
+    assert L.smoe_selftest_wait_timeout(1000, None, 272, None) == smoe.SMOE_ERR_INVALID_ARG
+    assert L.smoe_selftest_wait_timeout(1000, 12, 256, None) == smoe.SMOE_ERR_INVALID_ARG
+
+
 def test_workspace_checks():
     L = smoe.lib()
     c = smoe.config()

@@ -115,3 +115,20 @@ def test_expert_ffn_rejects_corrupt_offsets_and_still_runs_the_shared_expert():
                          packed, y, ws)
     torch.cuda.synchronize()
     assert torch.equal(y.view(torch.int16), good_y.view(torch.int16))
+
+
+def test_bounded_wait_times_out_and_the_context_stays_usable():
+    """The bounded mbarrier wait of the GEMM roles, run on a barrier nothing arrives at with a
+    50 ms limit: it gives up, records SMOE_ERR_TIMEOUT and returns; the layer then still runs."""
+    w, x, wr, bias, packed = device_inputs("tiny")
+    cfg = cfg_of(w)
+    ws = smoe.workspace(cfg, w.T)
+    elapsed = torch.zeros(1, dtype=torch.int64, device="cuda")
+    smoe.smoe_selftest_wait_timeout(50_000_000, elapsed, ws)
+    assert smoe.smoe_get_device_error(ws) == smoe.SMOE_ERR_TIMEOUT
+    assert 50_000_000 <= int(elapsed.item()) < 1_000_000_000
+    smoe.smoe_clear_device_error(ws)
+    out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+    smoe.smoe_forward(cfg, x, w.T, wr, bias, packed, out, ws)
+    assert smoe.smoe_get_device_error(ws) == 0
+    assert torch.isfinite(out.float()).all()
