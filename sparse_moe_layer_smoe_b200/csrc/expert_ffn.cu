@@ -174,6 +174,17 @@ __device__ __forceinline__ Unit decode_unit(int u, int units_per_tile, const int
     return Unit{g, u % units_per_tile, t & 0xFFFFF, nt};
 }
 
+#ifndef SMOE_REUSE_HINT
+#define SMOE_REUSE_HINT 1   // keep the weights of multi-tile groups in L2 (0: stream every weight tile)
+#endif
+// L2 policy of a unit's weight tiles. A group with several token tiles reads each weight tile
+// once per token tile, from neighbouring workers at about the same time: those tiles are kept
+// (evict-last) so that the later reads hit L2; a single-tile group's weights are read once and
+// streamed (evict-first).
+__device__ __forceinline__ uint64_t weight_policy(int rows, int nt, uint64_t stream_pol, uint64_t keep_pol) {
+    return (SMOE_REUSE_HINT && rows > nt) ? keep_pol : stream_pol;
+}
+
 // Unit of round i for worker w of W (snake order), or -1 when it lies past the last unit.
 __device__ __forceinline__ int snake_unit(int i, int w, int W, int total) {
     const int u = i * W + ((i & 1) ? W - 1 - w : w);
@@ -413,6 +424,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             const bool gather = p.row_token != nullptr && w.g < E;
             const CUtensorMap* bm = (w.g < E) ? &maps.act[gather ? 0 : ti] : &maps.sh[ti];
             const uint32_t tx = (uint32_t)(C::A_BYTES + w.nt * BK * 2);
+            const uint64_t pw = weight_policy(group_rows(w.g, E, p.T, offs), w.nt, pol_w, pol_a);
             // gather mode: this lane's chunks of 4 rows (chunk c = lane + 32 j) and their tokens
             int tok[8];
             const int nchunks = w.nt / 4;
@@ -438,11 +450,11 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 if (lane == 0) {
                     mbar_arrive_expect_tx(fb, tx);
                     if (MODE == MODE_ROUTER) {
-                        tma_load_2d(smem_u32(a_s), &maps.w, kg * BK, a_row, fb, pol_w);
+                        tma_load_2d(smem_u32(a_s), &maps.w, kg * BK, a_row, fb, pw);
                     } else {
                         int wx, wy;
                         weight_tile_xy<EK, TK>(w.g * MB + w.mb, kg, p.K, C::A_ROWS, wx, wy);
-                        tma_load_2d(smem_u32(a_s), &maps.w, wx, wy, fb, pol_w);
+                        tma_load_2d(smem_u32(a_s), &maps.w, wx, wy, fb, pw);
                     }
                     if (!gather) tma_load_2d(smem_u32(a_s + C::A_BYTES), bm, b_k * EK, b_row, fb, pol_a);
                 }
@@ -687,6 +699,7 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
             const int ti = tile_index(w.nt);
             const CUtensorMap* bm = (w.g < E) ? &maps.act[ti] : &maps.sh[ti];
             const uint32_t tx = (uint32_t)(2 * (C::A_BYTES + half * BK * 2));
+            const uint64_t pw = weight_policy(group_rows(w.g, E, p.T, offs), w.nt, pol_w, pol_a);
             for (int kb = 0; kb < KB; ++kb) {
                 if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag, true)) { ok = false; break; }
                 const uint32_t fb_local = smem_u32(&full[stage]);
@@ -695,7 +708,7 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
                 uint8_t* a_s = tiles + (size_t)stage * STAGE_B;
                 int wx, wy;
                 weight_tile_xy<EK, TK>(a_blk, kb, p.K, C::A_ROWS, wx, wy);
-                tma_load_2d_pair(smem_u32(a_s), &maps.w, wx, wy, fb_leader, pol_w);
+                tma_load_2d_pair(smem_u32(a_s), &maps.w, wx, wy, fb_leader, pw);
                 tma_load_2d_pair(smem_u32(a_s + C::A_BYTES), bm, kb * EK, b_row, fb_leader, pol_a);
                 armed |= 1u << stage;
                 armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
@@ -971,10 +984,13 @@ cudaError_t run_gemm_pair(const GemmMaps& maps, GemmParams p, int num_sms, cudaS
 
 // Largest token tile of a launch: the smallest power of two >= 1.25 x the mean rows per routed
 // expert, 16..256. Groups with fewer rows use smaller tiles inside the kernel.
+#ifndef SMOE_TILE_FACTOR
+#define SMOE_TILE_FACTOR 1.25
+#endif
 int choose_token_tile(const smoe_config_t& c, int64_t T) {
     const double mean = (double)T * c.top_k / c.n_experts;
     int nt = 16;
-    while (nt < SMOE_MAX_TOKEN_TILE && nt < 1.25 * mean) nt *= 2;
+    while (nt < SMOE_MAX_TOKEN_TILE && nt < SMOE_TILE_FACTOR * mean) nt *= 2;
     return nt;
 }
 
