@@ -38,9 +38,9 @@ namespace smoe {
 
 namespace {
 
-#ifndef SMOE_GEMM_BK
-#define SMOE_GEMM_BK 64          // K elements per pipeline stage (16, 32 or 64): 64 measured fastest
-#endif
+// K elements per pipeline stage of the bf16 kernels: 64 = one 128-byte swizzled row, the width
+// of a packed weight tile (stages of 32 and 16 measured slower and are not built).
+#define SMOE_GEMM_BK 64
 #ifndef SMOE_MAX_TOKEN_TILE
 #define SMOE_MAX_TOKEN_TILE 256  // cap on the token tile (a tuning constant)
 #endif
@@ -103,7 +103,7 @@ struct GemmCfg {
     static constexpr int A_ROWS = DUAL ? 256 : 128;       // gate 128 + up 128, or 128
     static constexpr int A_BYTES = A_ROWS * SW;
     static constexpr int UP_OFFSET = 128 * SW;            // up rows inside the A tile
-    static_assert(BK == 16 || BK == 32 || BK == 64, "stage K width");
+    static_assert(BK == 64, "stage K width: one 128-byte row of a packed tile");
 };
 
 __host__ __device__ inline int stage_bytes(bool dual, int bk, int nt_max) {
