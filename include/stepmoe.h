@@ -244,8 +244,9 @@ SMOE_API smoe_status_t smoe_pack_weights_fp8(const smoe_config_t* cfg, const smo
 /* Workspace bytes of smoe_forward_fp8 for T tokens (smoe_forward's plus the e4m3 activations). */
 SMOE_API smoe_status_t smoe_workspace_bytes_fp8(const smoe_config_t* cfg, int64_t T, size_t* bytes);
 
-/* The whole layer with e4m3 experts: route (fp32, as smoe_forward) -> quantise x per token ->
- * permute -> gate/up (e4m3 tensor cores) -> quantise h per row -> down -> combine. Arguments as
+/* The whole layer with e4m3 experts: route (fp32, as smoe_forward; its top-k kernel also
+ * quantises x per token) -> permute -> gate/up (e4m3 tensor cores) -> quantise h per row ->
+ * down -> combine. Arguments as
  * smoe_forward, with packed_fp8 from smoe_pack_weights_fp8 and a workspace of at least
  * smoe_workspace_bytes_fp8(cfg, T) bytes. */
 SMOE_API smoe_status_t smoe_forward_fp8(const smoe_config_t* cfg, const smoe_bf16_t* x, int64_t T,

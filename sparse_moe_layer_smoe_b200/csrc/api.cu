@@ -372,8 +372,11 @@ smoe_status_t forward_impl(const smoe_config_t* c, const smoe_bf16_t* x, int64_t
     uint16_t* y = at<uint16_t>(ws, L.y);
     float* conf = diag != nullptr ? diag->token_confidence : nullptr;
     float* row_norm = diag != nullptr ? at<float>(ws, L.row_norm) : nullptr;
+    // e4m3: the top-k kernel also quantises x per token
+    uint8_t* x_q = fp8 ? at<uint8_t>(ws, L.x_q) : nullptr;
+    float* s_x = fp8 ? at<float>(ws, L.s_x) : nullptr;
     cudaError_t e = launch_route(*c, x, T, w_router, bias, idx, w, nullptr, at<float>(ws, L.route_partials), err,
-                                 sms, s, true, conf);
+                                 sms, s, true, conf, x_q, s_x);
     // small token tiles: routed rows are gathered from x inside the expert GEMM (no permuted
     // copy); large tiles: one gather kernel writes x_perm and the GEMM loads whole tiles
     const bool gather = choose_token_tile(*c, T) <= kGatherMaxTile;
@@ -386,11 +389,8 @@ smoe_status_t forward_impl(const smoe_config_t* c, const smoe_bf16_t* x, int64_t
             e = launch_expert_ffn(*c, x, x_perm, row_token, offsets, T, packed, y, at<uint16_t>(ws, L.ffn_h), err, sms,
                                   s);
     } else {
-        // e4m3: x quantised per token; the permuted copy (large tiles) is of the e4m3 rows, moved
-        // by the same gather kernel as 2-byte pairs
-        uint8_t* x_q = at<uint8_t>(ws, L.x_q);
-        float* s_x = at<float>(ws, L.s_x);
-        if (e == cudaSuccess) e = launch_quantize_rows(x, T, c->hidden, x_q, s_x, K_QUANT_X, s);
+        // e4m3: x was quantised per token by the top-k kernel; the permuted copy (large tiles) is
+        // of the e4m3 rows, moved by the same gather kernel as 2-byte pairs
         if (e == cudaSuccess)
             e = launch_permute(*c, idx, T, gather ? nullptr : reinterpret_cast<const uint16_t*>(x_q),
                                at<int32_t>(ws, L.counts), offsets, perm_row, row_token, x_perm,

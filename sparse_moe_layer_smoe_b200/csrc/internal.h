@@ -88,7 +88,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, const float* wr, const float* bias,
                          int32_t* topk_idx, float* topk_w, float* logits_opt, float* partials, int32_t* err,
-                         int num_sms, cudaStream_t s, bool allow_tc = true, float* conf_opt = nullptr);
+                         int num_sms, cudaStream_t s, bool allow_tc = true, float* conf_opt = nullptr,
+                         uint8_t* x_q_opt = nullptr, float* s_x_opt = nullptr);   // x_q: e4m3 x per token
 
 cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* w_split, int e_pad, int E,
                                float* logits, int nt, int ksplit, int num_sms, cudaStream_t s);

@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "quant.cuh"
 
 namespace smoe {
 
@@ -164,7 +165,8 @@ template <int NPL>
 __global__ void __launch_bounds__(256)
 router_topk_kernel(const float* __restrict__ part, int splits, const float* __restrict__ bias, int T, int E, int k,
                    float scale, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-                   float* __restrict__ logits_out, float* __restrict__ conf_out) {
+                   float* __restrict__ logits_out, float* __restrict__ conf_out, const uint16_t* __restrict__ x,
+                   int H, uint8_t* __restrict__ x_q, float* __restrict__ s_x) {
     pdl_wait();
     pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
@@ -262,6 +264,12 @@ router_topk_kernel(const float* __restrict__ part, int splits, const float* __re
         topk_w[(size_t)t * k + lane] = scale * (s_sel / sum);
     }
     if (conf_out != nullptr && lane == 0) conf_out[t] = sum / (float)k;   // routing confidence
+    if (x_q != nullptr) {
+        // e4m3 layer: this token's row of x quantised here, saving a launch
+        uint2* dst = reinterpret_cast<uint2*>(x_q + (size_t)t * H);
+        const float sc = quantize_row_warp(x + (size_t)t * H, H, [&](int v, uint2 c) { dst[v] = c; });
+        if (lane == 0) s_x[t] = sc;
+    }
 }
 
 // W_split[e][p*H + h] = piece p (0 = hi, 1 = mid, 2 = lo) of W_r[e][h]: hi = bf16(w),
@@ -324,12 +332,13 @@ cudaError_t launch_logits(const uint16_t* x, int64_t T, const float* wr, int E, 
 
 template <int NPL>
 cudaError_t launch_topk(const float* part, int splits, const float* bias, int64_t T, int E, int k, float scale,
-                        int32_t* idx, float* w, float* logits, float* conf, cudaStream_t s) {
+                        int32_t* idx, float* w, float* logits, float* conf, const uint16_t* x, int H, uint8_t* x_q,
+                        float* s_x, cudaStream_t s) {
     const int warps = 8;
     {
         LaunchTimer lt(K_ROUTER_TOPK, s);
         return launch_pdl(router_topk_kernel<NPL>, dim3((unsigned)((T + warps - 1) / warps)), dim3(warps * 32), 0, s,
-                          part, splits, bias, (int)T, E, k, scale, idx, w, logits, conf);
+                          part, splits, bias, (int)T, E, k, scale, idx, w, logits, conf, x, H, x_q, s_x);
     }
 }
 
@@ -391,7 +400,8 @@ RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms, bool allo
 
 cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, const float* wr, const float* bias,
                          int32_t* topk_idx, float* topk_w, float* logits_opt, float* partials, int32_t* err,
-                         int num_sms, cudaStream_t s, bool allow_tc, float* conf_opt) {
+                         int num_sms, cudaStream_t s, bool allow_tc, float* conf_opt, uint8_t* x_q_opt,
+                         float* s_x_opt) {
     (void)err;
     const RouterPlan p = router_plan(c, T, num_sms, allow_tc);
     const int E = c.n_experts, H = c.hidden;
@@ -420,13 +430,13 @@ cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, c
     if (e != cudaSuccess) return e;
     const int npl = (E + 31) / 32;
     if (npl <= 4)
-        e = launch_topk<4>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, s);
+        e = launch_topk<4>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, x, H, x_q_opt, s_x_opt, s);
     else if (npl <= 9)
-        e = launch_topk<9>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, s);
+        e = launch_topk<9>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, x, H, x_q_opt, s_x_opt, s);
     else if (npl <= 16)
-        e = launch_topk<16>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, s);
+        e = launch_topk<16>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, x, H, x_q_opt, s_x_opt, s);
     else
-        e = launch_topk<32>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, s);
+        e = launch_topk<32>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, x, H, x_q_opt, s_x_opt, s);
     if (e == cudaSuccess) launches_add(n);
     return e;
 }
