@@ -4,7 +4,8 @@
   experts of the tiny layer and of the Step shape (the same warp routine quantises x and h);
 * smoe_forward_fp8: the layer vs the oracle's e4m3 layer within the layer tolerances (relative
   Frobenius <= 1e-2, max |err| <= 2e-2 max|ref|): all tokens of the tiny layer, sampled tokens
-  (spike rows included) at decode (gather mode), MTP and prefill (CTA pairs, permuted e4m3 rows);
+  (spike rows included) at decode (gather mode), MTP, prefill and the Zipf-skewed batch (CTA
+  pairs, permuted e4m3 rows; skewed mixes 1-row and multi-tile groups);
   the quantisation error against the bf16 oracle is printed for reference;
 * deterministic: two calls give the same bits.
 """
@@ -99,7 +100,7 @@ def _oracle_rows(name, rows, w):
     return ref8, ref16
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode", "mtp", "prefill"])
+@pytest.mark.parametrize("name", ["tiny", "decode", "mtp", "prefill", "skewed"])
 def test_forward_fp8_parity(name):
     w, out = _forward_fp8(name)
     r = host_route(name)
