@@ -247,12 +247,12 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
         const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
         uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * H);
         int c = lane;
-        for (; c + 96 < vec; c += 128) {   // four 16-byte vectors in flight per lane
-            const uint4 a = src[c], b = src[c + 32], d = src[c + 64], e = src[c + 96];
-            dst[c] = a;
-            dst[c + 32] = b;
-            dst[c + 64] = d;
-            dst[c + 96] = e;
+        for (; c + 224 < vec; c += 256) {   // eight 16-byte vectors in flight per lane
+            uint4 v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = __ldg(src + c + 32 * i);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[c + 32 * i] = v[i];
         }
         for (; c < vec; c += 32) dst[c] = src[c];
     }

@@ -363,11 +363,12 @@ RouterPlan router_plan(const smoe_config_t& c, int64_t T, int num_sms, bool allo
         p.e_pad = (E + 127) / 128 * 128;
         const int mb = p.e_pad / 128;
         p.nt = 256;
-        while (p.nt > 64 && ((T + p.nt - 1) / p.nt) * mb * 3 < num_sms) p.nt /= 2;
+        const int64_t enough = (3 * (int64_t)num_sms) / 4;   // one round of units on 3/4 of the SMs
+        while (p.nt > 64 && ((T + p.nt - 1) / p.nt) * mb * 3 < enough) p.nt /= 2;
         // K = the three bf16 pieces of W_r, each in m equal ranges: one partial per range,
         // summed in order by the top-k kernel (m grows until the units cover the SMs)
         int m = 1;
-        while (m < 4 && c.hidden % (128 * m) == 0 && ((T + p.nt - 1) / p.nt) * mb * 3 * m < num_sms) m *= 2;
+        while (m < 4 && c.hidden % (128 * m) == 0 && ((T + p.nt - 1) / p.nt) * mb * 3 * m < enough) m *= 2;
         p.splits = 3 * m;
         const size_t logit_b = ((size_t)p.splits * T * E * 4 + 255) / 256 * 256;
         p.scratch_bytes = logit_b + (size_t)p.e_pad * 3 * c.hidden * 2;
