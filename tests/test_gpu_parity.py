@@ -10,7 +10,8 @@ seeded inputs, on all five workloads, at their full sizes.
   tiny layer, sampled rows of every kind at the Step shape);
 * combine: fed seeded bf16 rows and the oracle's weights, vs the fp64 formula within 1 bf16 ulp;
 * forward (the launch configuration bench.py times): the whole layer vs the oracle, dense-masked
-  for tiny and decode, sparse on sampled tokens (incl. near-tie and spike rows) otherwise.
+  for tiny and decode, sparse on sampled tokens (incl. near-tie and spike rows) otherwise; and a
+  degenerate routing collapse (every token to the same 8 experts) on both GEMM kernels.
 """
 import numpy as np
 import pytest
@@ -352,3 +353,37 @@ def test_forward_ragged_token_counts(T):
     ref = oracle.moe_sparse(x64, r, HostExperts(w), w.E)
     keep = ~r.near_tie   # a near tie may resolve to another valid selection; checked in test_route_parity
     assert_close(bf16_tensor_to_f64(out)[keep], ref[keep], f"tiny T={T}")
+
+
+@pytest.mark.parametrize("T", [512, 2048])
+def test_forward_routing_collapse(T):
+    """Degenerate routing (the routing collapse that the loss-free balancing bias is there to
+    prevent, pushed to its limit): a bias of +20 on 8 experts sends every token to the same 8, so
+    8 groups hold all T*k routed rows, in many token tiles each, and the other 280 are empty
+    (single-CTA kernel with 16-row tiles at T=512, CTA pairs with 128-row tiles at T=2048)."""
+    w0 = synth.WORKLOADS["mtp"]
+    w = synth.Workload("collapse", T, w0.H, w0.E, w0.k, w0.I, w0.Is)
+    cfg = cfg_of(w)
+    _, _, wr, _, packed = device_inputs("mtp")
+    hot = np.array([3, 17, 50, 97, 144, 191, 238, 285])
+    bias_h = np.zeros(w.E, dtype=np.float32)
+    bias_h[hot] = 20.0
+    bias = torch.from_numpy(bias_h).cuda()
+    x = synth.dev_x(w)
+    out = torch.empty(T, w.H, dtype=torch.bfloat16, device="cuda")
+    smoe.smoe_forward(cfg, x, T, wr, bias, packed, out, _ws(cfg, T, forward=True))
+    idx = torch.empty(T, w.k, dtype=torch.int32, device="cuda")
+    wt = torch.empty(T, w.k, dtype=torch.float32, device="cuda")
+    ws = _ws(cfg, T)
+    smoe.smoe_route(cfg, x, T, wr, bias, idx, wt, None, ws)
+    assert smoe.smoe_get_device_error(ws) == 0
+    assert np.array_equal(np.sort(idx.cpu().numpy(), axis=1), np.tile(hot, (T, 1)))
+    x64 = oracle.bf16_to_f64(synth.host_x(w))
+    r = oracle.route(x64, oracle.f32_to_f64(synth.host_w_router(w)), bias_h.astype(np.float64), w.k, w.route_scale)
+    assert np.array_equal(np.sort(r.idx, axis=1), np.tile(hot, (T, 1)))
+    rows = sorted({0, T - 1, *RNG.integers(0, T, 6).tolist()})
+    sub = oracle.Route(r.logits[rows], r.s[rows], r.bhat[rows], r.idx[rows], r.w[rows], r.gap[rows])
+    ref = oracle.moe_sparse(x64[rows], sub, HostExperts(w, cap=9), w.E)
+    fro, mx = assert_close(bf16_tensor_to_f64(out)[rows], ref, f"collapse T={T} forward (sampled tokens)")
+    assert torch.isfinite(out.float()).all()
+    print(f"collapse T={T}: rows={len(rows)} rel_fro={fro:.2e} rel_max={mx:.2e}")
