@@ -24,6 +24,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -92,10 +93,15 @@ def measured_peaks():
 
 
 def source_sha(paths) -> str:
+    """Hash of the code of the given sources with comments and whitespace removed, so that an
+    edit of comments alone keeps the committed counters valid."""
     h = hashlib.sha256()
     for p in paths:
-        with open(os.path.join(REPO, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(REPO, p), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -17,9 +17,9 @@
 // Token tile per group: the smallest power of two >= the group's row count, between 16 and a
 // launch-wide maximum NT_MAX (so an expert with 2 tokens runs N=16 MMAs while a hot expert with
 // 1000 tokens runs N=256 tiles). One TMA tensor map per tile height loads exactly that box.
-// Work unit = (token tile (group, nb), 128-feature block mb). The token tiles are sorted by the
-// MMA columns they run (largest first) and the units dealt to the CTAs in snake order (static
-// persistent schedule, grid = #SMs): see the work table below.
+// Work unit = (token tile (group, nb), 128-feature block mb). The token tiles are listed in
+// group order and the units dealt to the CTAs in snake order (static persistent schedule,
+// grid = #SMs): see the work table below.
 //
 // Roles (192 threads): warp 0 lane 0 issues TMA loads into an S-stage ring of BK-wide K slices
 // (BK = 64: 128-byte swizzled rows; the ring fills the 227 KB of shared memory);
@@ -601,7 +601,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
 // and accumulates into both CTAs' TMEM (128 rows each). Per SM this moves 25-30% fewer operand
 // bytes through shared memory per MMA than the single-CTA kernel, whose token tile every SM
 // loads in full. Work unit = (token tile, 256-feature block), dealt to the pairs in the same
-// cost-sorted snake order as the single-CTA kernel's units.
+// snake order as the single-CTA kernel's units.
 //
 // Signals: both CTAs' loads complete on the first CTA's stage barrier (it arms the expected
 // bytes of both); the first CTA's MMA thread commits stage-free and accumulator-ready to each
