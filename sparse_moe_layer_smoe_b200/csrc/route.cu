@@ -161,16 +161,29 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-template <int NPL>
+// QX: 0 = no x quantisation (bf16 layer); 1 = quantise x before the dependency wait (the router
+// kernel before it is the CUDA-core one, beside which this grid's CTAs can already run);
+// 2 = quantise x at the end (after a tensor-core router GEMM, which leaves no room to co-run,
+// and where the first variant's extra registers cost occupancy).
+template <int NPL, int QX>
 __global__ void __launch_bounds__(256)
 router_topk_kernel(const float* __restrict__ part, int splits, const float* __restrict__ bias, int T, int E, int k,
                    float scale, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                    float* __restrict__ logits_out, float* __restrict__ conf_out, const uint16_t* __restrict__ x,
                    int H, uint8_t* __restrict__ x_q, float* __restrict__ s_x) {
-    pdl_wait();
-    pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (QX == 1 && t < T) {
+        // e4m3 layer: this token's row of x quantised here, saving a launch. x does not come
+        // from the router, so this runs before the wait, while the router kernel still works:
+        // this grid only launches once the router kernel has passed its own wait, i.e. after
+        // every kernel of the previous layer call (the last readers of x_q) has completed.
+        uint2* dst = reinterpret_cast<uint2*>(x_q + (size_t)t * H);
+        const float sc = quantize_row_warp(x + (size_t)t * H, H, [&](int v, uint2 c) { dst[v] = c; });
+        if (lane == 0) s_x[t] = sc;
+    }
+    pdl_wait();
+    pdl_launch_dependents();
     if (t >= T) return;
 
     // logits: the K-split partials added in split order 0, 1, 2, ... (the order is fixed, so the
@@ -264,8 +277,7 @@ router_topk_kernel(const float* __restrict__ part, int splits, const float* __re
         topk_w[(size_t)t * k + lane] = scale * (s_sel / sum);
     }
     if (conf_out != nullptr && lane == 0) conf_out[t] = sum / (float)k;   // routing confidence
-    if (x_q != nullptr) {
-        // e4m3 layer: this token's row of x quantised here, saving a launch
+    if (QX == 2) {
         uint2* dst = reinterpret_cast<uint2*>(x_q + (size_t)t * H);
         const float sc = quantize_row_warp(x + (size_t)t * H, H, [&](int v, uint2 c) { dst[v] = c; });
         if (lane == 0) s_x[t] = sc;
@@ -333,12 +345,19 @@ cudaError_t launch_logits(const uint16_t* x, int64_t T, const float* wr, int E, 
 template <int NPL>
 cudaError_t launch_topk(const float* part, int splits, const float* bias, int64_t T, int E, int k, float scale,
                         int32_t* idx, float* w, float* logits, float* conf, const uint16_t* x, int H, uint8_t* x_q,
-                        float* s_x, cudaStream_t s) {
+                        float* s_x, bool after_tc_router, cudaStream_t s) {
     const int warps = 8;
+    const dim3 grid((unsigned)((T + warps - 1) / warps)), block(warps * 32);
     {
         LaunchTimer lt(K_ROUTER_TOPK, s);
-        return launch_pdl(router_topk_kernel<NPL>, dim3((unsigned)((T + warps - 1) / warps)), dim3(warps * 32), 0, s,
-                          part, splits, bias, (int)T, E, k, scale, idx, w, logits, conf, x, H, x_q, s_x);
+        if (x_q == nullptr)
+            return launch_pdl(router_topk_kernel<NPL, 0>, grid, block, 0, s, part, splits, bias, (int)T, E, k, scale,
+                              idx, w, logits, conf, x, H, x_q, s_x);
+        if (!after_tc_router)
+            return launch_pdl(router_topk_kernel<NPL, 1>, grid, block, 0, s, part, splits, bias, (int)T, E, k, scale,
+                              idx, w, logits, conf, x, H, x_q, s_x);
+        return launch_pdl(router_topk_kernel<NPL, 2>, grid, block, 0, s, part, splits, bias, (int)T, E, k, scale, idx,
+                          w, logits, conf, x, H, x_q, s_x);
     }
 }
 
@@ -431,13 +450,13 @@ cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, c
     if (e != cudaSuccess) return e;
     const int npl = (E + 31) / 32;
     if (npl <= 4)
-        e = launch_topk<4>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, x, H, x_q_opt, s_x_opt, s);
+        e = launch_topk<4>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, x, H, x_q_opt, s_x_opt, p.tc, s);
     else if (npl <= 9)
-        e = launch_topk<9>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, x, H, x_q_opt, s_x_opt, s);
+        e = launch_topk<9>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, x, H, x_q_opt, s_x_opt, p.tc, s);
     else if (npl <= 16)
-        e = launch_topk<16>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, x, H, x_q_opt, s_x_opt, s);
+        e = launch_topk<16>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, x, H, x_q_opt, s_x_opt, p.tc, s);
     else
-        e = launch_topk<32>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, x, H, x_q_opt, s_x_opt, s);
+        e = launch_topk<32>(partials, p.splits, bias, T, E, c.top_k, c.route_scale, topk_idx, topk_w, logits_opt, conf_opt, x, H, x_q_opt, s_x_opt, p.tc, s);
     if (e == cudaSuccess) launches_add(n);
     return e;
 }
