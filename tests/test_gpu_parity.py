@@ -304,8 +304,9 @@ def test_forward_parity_sampled(name):
     print(f"{name}: forward rows={len(rows)} rel_fro={fro:.2e} rel_max={mx:.2e} near_ties={int(r.near_tie.sum())}")
 
 
-def test_forward_is_deterministic_and_matches_per_call_chain():
-    name = "mtp"
+@pytest.mark.parametrize("name", ["mtp", "decode"])
+def test_forward_is_deterministic_and_matches_per_call_chain(name):
+    """smoe_forward twice (same bits), and the same bits as chaining the four calls."""
     w, out1, _ = _forward(name)
     _, out2, _ = _forward(name)
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
