@@ -6,15 +6,18 @@
 
 A step is one pass of the whole layer (route -> permute -> expert FFNs -> combine, one
 smoe_forward call) over one batch of seeded synthetic tokens, weights resident in HBM. The
-default workload is the decode batch (T=64, hidden 4096, 288 experts top-8, intermediate 1280,
-one shared expert). Prints one JSON line on rank 0.
+headline workload is the decode batch (T=64, hidden 4096, 288 experts top-8, intermediate 1280,
+one shared expert); the same run also times the prefill (T=8192), skewed (T=4096, Zipf
+popularity, 16 dead experts) and MTP-verify (T=512, activation spikes) batches on the same
+weights and reports each under "workloads" with its own roofline, step-time spread, expert
+statistics and routing check. Prints one JSON line on rank 0.
 
 Multi-GPU: the layer does not shard across GPUs here (no exchange step), so N GPUs run N
 independent replicas of the same workload, launched one process per GPU by torchrun; the
 timed region is bracketed by barriers and the slowest rank's time is reported (value = all
 ranks' tokens / that time).
 
---impl reference times the CPU fp64 oracle as it stands on the host cores, on a bounded
+--impl reference times the C++ fp64 oracle as it stands on the host cores, on a bounded
 sample of the same workload (there is no other reference implementation of this layer).
 """
 from __future__ import annotations
@@ -45,7 +48,11 @@ def parse_args(argv=None):
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
-    p.add_argument("--workload", default="decode")
+    p.add_argument("--workload", default="decode", help="the headline workload (value, e2e, roofline)")
+    p.add_argument("--workloads", default="decode,prefill,skewed,mtp",
+                   help="comma list of further workloads of the same layer shape timed in the same run and "
+                        "reported under 'workloads' ('none': the headline only)")
+    p.add_argument("--pct-steps", type=int, default=50, help="steps of the per-step spread pass (p10/p50/p90)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=4)
@@ -133,7 +140,7 @@ class ClockSampler:
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.005):
+    def __init__(self, index: int, period_s: float = 0.001):
         self.samples, self.reasons, self.max_mhz = [], 0, None
         self.period = period_s
         self._stop = threading.Event()
@@ -177,6 +184,9 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------ CPU oracle leg
+# The oracle (the C++ fp64 program, test infrastructure) is run here only: timed as the CPU
+# baseline and the reference arm, and used untimed to count near-tie tokens and to check the
+# GPU's selections against its fp64 router.
 def oracle_sample(w, n_tokens: int):
     """Inputs of the oracle for the first n_tokens tokens: fp64 x, router, bias and fp64 weights of
     every expert those tokens select (prepared before any timing)."""
@@ -194,36 +204,60 @@ def oracle_sample(w, n_tokens: int):
     return x64, wr64, bias, experts
 
 
-def oracle_step(w, x64, wr64, bias, experts):
+def oracle_forward_seconds(w, x64, wr64, bias, experts, repeats: int) -> float:
+    """Seconds of `repeats` oracle passes (route + sparse layer) over x64, timed inside the C++
+    oracle with std::chrono::steady_clock."""
     import oracle
-    r = oracle.route(x64, wr64, bias, w.k, w.route_scale)
-    return oracle.moe_sparse(x64, r, lambda e: experts[e], w.E)
+    _, sec = oracle.cpp.forward_timed(x64, wr64, bias, w.k, w.route_scale, lambda e: experts[e], w.E, repeats,
+                                      w.swiglu_limit, w.swiglu_limit_shared)
+    return sec
 
 
-def blas_threads() -> int:
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
-        if n:
-            return int(max(n))
-    except Exception:
-        pass
-    return os.cpu_count() or 1
+def oracle_threads() -> int:
+    import oracle
+    return oracle.cpp.threads()
 
 
 def cpu_baseline(w, n_tokens: int, min_seconds: float):
     x64, wr64, bias, experts = oracle_sample(w, n_tokens)
-    oracle_step(w, x64, wr64, bias, experts)   # warm-up
-    done, t0 = 0, time.perf_counter()
-    while True:
-        oracle_step(w, x64, wr64, bias, experts)
-        done += x64.shape[0]
-        el = time.perf_counter() - t0
-        if el >= min_seconds:
-            break
-    return {"value": done / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"first {x64.shape[0]} tokens of the {w.name} batch (fp64 numpy oracle, sparse mode; fp64 "
-                      f"weights of their {len(experts)} experts prepared untimed), repeated for {el:.1f} s"}
+    one = oracle_forward_seconds(w, x64, wr64, bias, experts, 1)   # also the warm-up
+    repeats = max(1, int(min_seconds / max(one, 1e-6)))
+    el = oracle_forward_seconds(w, x64, wr64, bias, experts, repeats)
+    done = repeats * x64.shape[0]
+    return {"value": done / el, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "implementation": "C++17 fp64 oracle (oracle/smoe_oracle.cpp: plain loops, std::sort, std::thread)",
+            "sample": f"first {x64.shape[0]} tokens of the {w.name} batch, {repeats} passes of route + sparse layer "
+                      f"timed with std::chrono in the C++ oracle ({el:.1f} s); fp64 weights of their "
+                      f"{len(experts)} experts prepared untimed"}
+
+
+def routing_check(w, gpu_idx):
+    """The GPU's selections against the oracle's fp64 router on the whole batch (untimed):
+    near-tie tokens (8th/9th biased-score gap < 1e-5), selections that differ outside near ties
+    (must be 0), and tokens whose selected order differs from the oracle's — within the 1e-5
+    band, where fp32 rounding may swap two experts, and beyond it (must be 0)."""
+    import numpy as np
+
+    import oracle
+    import synth
+    r = oracle.route(oracle.bf16_to_f64(synth.host_x(w)), oracle.f32_to_f64(synth.host_w_router(w)),
+                     synth.host_bias(w).astype(np.float64), w.k, w.route_scale)
+    near = r.near_tie
+    differs = np.array([set(a) != set(b) for a, b in zip(gpu_idx.tolist(), r.idx.tolist())])
+    order_in_band = order_beyond = 0
+    for t in np.nonzero(~differs & ~near)[0]:
+        g = gpu_idx[t]
+        if np.array_equal(g, r.idx[t]):
+            continue
+        b = r.bhat[t, g]
+        if np.all(b[:-1] >= b[1:] - oracle.NEAR_TIE_EPS):
+            order_in_band += 1
+        else:
+            order_beyond += 1
+    return {"near_tie_tokens": int(near.sum()), "selection_differs_outside_near_ties": int((differs & ~near).sum()),
+            "selection_differs_at_near_ties": int((differs & near).sum()),
+            "order_differs_within_1e-5": int(order_in_band), "order_differs_beyond_1e-5": int(order_beyond),
+            "oracle": "C++ fp64 router"}
 
 
 def run_reference(args):
@@ -235,19 +269,21 @@ def run_reference(args):
     x64, wr64, bias, experts = oracle_sample(w, args.cpu_sample_tokens)
     n = x64.shape[0]
     for i in range(args.warmup):
-        oracle_step(w, x64[i % n:i % n + 1], wr64, bias, experts)
-    t0 = time.perf_counter()
+        oracle_forward_seconds(w, x64[i % n:i % n + 1], wr64, bias, experts, 1)
+    el = 0.0
     for i in range(args.steps):
-        oracle_step(w, x64[i % n:i % n + 1], wr64, bias, experts)
-    el = time.perf_counter() - t0
+        el += oracle_forward_seconds(w, x64[i % n:i % n + 1], wr64, bias, experts, 1)
     value = args.steps / el
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                             "implementation": "C++17 fp64 oracle (oracle/smoe_oracle.cpp: plain loops, std::sort, "
+                                               "std::thread)",
                              "sample": f"one token per step, cycling over the first {n} tokens of the {w.name} "
-                                       f"batch; fp64 weights of their {len(experts)} experts prepared untimed"},
+                                       f"batch, each step timed with std::chrono in the C++ oracle; fp64 weights "
+                                       f"of their {len(experts)} experts prepared untimed"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -262,48 +298,63 @@ def workload_config(w):
             "l2": "inputs larger than L2: every step streams the active experts' bf16 weights (GBs) from HBM"}
 
 
-def run_ours(args):
+def percentiles(v):
+    import numpy as np
+    a = np.asarray(v, dtype=np.float64)
+    return {"p10": float(np.percentile(a, 10)), "p50": float(np.percentile(a, 50)),
+            "p90": float(np.percentile(a, 90)), "steps": int(a.size)}
+
+
+def kernel_bytes_flops(w, touched: int, fp8: bool):
+    """Algorithmic bytes and flops of one launch of each expert GEMM: the weights of the touched
+    experts and the shared one, the GEMM's input activations and its output."""
+    H, I, T, k = w.H, w.I, w.T, w.k
+    wb = 1 if fp8 else 2   # bytes per weight (e4m3 or bf16); e4m3 adds one fp32 scale per weight row
+    ab = 1 if fp8 else 2   # bytes per GEMM input activation
+    rows = T * k + T
+    gate_up = (touched + 1) * 2 * I * (H * wb + (4 if fp8 else 0)) + rows * H * ab + rows * I * 2
+    down = (touched + 1) * H * (I * wb + (4 if fp8 else 0)) + rows * I * ab + rows * H * 2
+    return ({"expert_gateup": gate_up, "expert_down": down},
+            {"expert_gateup": 2.0 * rows * 2 * I * H, "expert_down": 2.0 * rows * H * I})
+
+
+def measure(smoe, w, packed, args, dev, headline: bool):
+    """Time one workload: the device-resident steps (value), per-kernel split, per-step spread and
+    the end-to-end steps from pinned host buffers. Returns (entry, GPU top-k indices)."""
     import torch
 
-    import sparse_moe_layer_smoe_b200 as smoe
     import synth
-
-    rank, local, world = dist_env()
-    torch.cuda.set_device(local)
-    init_dist(world, "nccl")
-    dev = torch.device("cuda", local)
-    w = synth.WORKLOADS[args.workload]
+    fp8 = args.fp8
     cfg = smoe.config(w.H, w.E, w.k, w.I, w.Is, w.route_scale, w.swiglu_limit, w.swiglu_limit_shared)
-    T = w.T
-
+    T, E = w.T, w.E
+    rank, local, world = dist_env()
     x = synth.dev_x(w, device=dev)
     wr, bias = synth.dev_router(w, device=dev)
-    experts = synth.dev_experts(w, device=dev)
-    packed = smoe.pack_weights_fp8(cfg, *experts) if args.fp8 else smoe.pack_weights(cfg, *experts)
-    torch.cuda.synchronize()
-    del experts
-    torch.cuda.empty_cache()
-    ws = smoe.workspace(cfg, T, device=dev, fp8=args.fp8)
+    ws = smoe.workspace(cfg, T, device=dev, fp8=fp8)
     out = torch.empty(T, w.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
     diag = smoe.diag_buffers(cfg, T, device=dev) if args.diag else None
 
     def forward(x_):
-        if args.fp8:
+        if fp8:
             smoe.smoe_forward_fp8(cfg, x_, T, wr, bias, packed, out, ws)
         elif diag is None:
             smoe.smoe_forward(cfg, x_, T, wr, bias, packed, out, ws)
         else:
             smoe.smoe_forward_diag(cfg, x_, T, wr, bias, packed, out, diag, ws)
 
-    # routing statistics of this batch (for the algorithmic byte count): experts touched
+    # routing of this batch on the GPU (for the algorithmic byte count and the expert statistics)
     idx = torch.empty(T, w.k, dtype=torch.int32, device=dev)
     wt = torch.empty(T, w.k, dtype=torch.float32, device=dev)
     sws = smoe.workspace(cfg, T, forward=False, device=dev)
     smoe.smoe_route(cfg, x, T, wr, bias, idx, wt, None, sws)
-    counts = torch.bincount(idx.view(-1).long(), minlength=w.E)
-    touched = int((counts > 0).sum().item())
+    counts = torch.bincount(idx.view(-1).long(), minlength=E).cpu()
+    gpu_idx = idx.cpu().numpy()
     del sws
+    touched = int((counts > 0).sum().item())
+    live = counts[counts > 0]
+    experts = {"touched": touched, "dead": E - touched, "max_count": int(counts.max().item()),
+               "min_count_live": int(live.min().item()) if touched else 0, "mean_count": T * w.k / E}
 
     # ---- device-resident timing (value)
     for _ in range(args.warmup):
@@ -320,8 +371,18 @@ def run_ours(args):
         ev1.record(stream)
         torch.cuda.synchronize()
     barrier()
-    ms = ev0.elapsed_time(ev1) / args.steps
-    ms = max_over_ranks(ms, dev)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
+
+    # ---- per-step spread, in a pass of its own: an event between steps keeps the next step's
+    # first kernel from starting under the previous step's last one
+    n_pct = max(args.steps, args.pct_steps)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_pct + 1)]
+    evs[0].record(stream)
+    for i in range(n_pct):
+        forward(x)
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    spread = percentiles([evs[i].elapsed_time(evs[i + 1]) for i in range(n_pct)])
 
     # ---- per-kernel split, in a separate pass: the library records CUDA events around each of
     # its launches, which serialises the kernels (the timed steps above let each kernel launch
@@ -334,7 +395,7 @@ def run_ours(args):
     ktimes = smoe.smoe_timing_end()
     err = smoe.smoe_get_device_error(ws)
     if err != 0:
-        raise RuntimeError(f"device error word {smoe.STATUS.get(err, err)}")
+        raise RuntimeError(f"{w.name}: device error word {smoe.STATUS.get(err, err)}")
 
     # ---- end to end through the C-ABI from pinned host buffers (copies inside the region)
     x_host = x.cpu().pin_memory()
@@ -360,57 +421,103 @@ def run_ours(args):
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
 
-    # ---- roofline of the dominant kernel
+    # ---- rooflines: the layer, and its dominant kernel
     peaks, peak_src = measured_peaks()
+    tc_mult = 2.0 if fp8 else 1.0   # e4m3 peak = the measured bf16 peak x 2 (nominal 4.5 / 2.25 PFLOP/s)
+    tc_sus, tc_burst = peaks["bf16_tflops_sustained"] * tc_mult, peaks["bf16_tflops"] * tc_mult
+    H, I, k = w.H, w.I, w.k
+    wb = 1 if fp8 else 2
+    layer_bytes = (touched + 1) * 3 * H * I * wb + E * H * 4 + 2 * T * H * 2
+    layer_flops = 2.0 * T * (k + 1) * 3 * H * I
+    s = ms / 1e3
+    layer = {"hbm_gbs": layer_bytes / s / 1e9, "hbm_frac": layer_bytes / s / 1e9 / peaks["hbm_gbs"],
+             "tflops": layer_flops / s / 1e12, "tflops_frac_sustained": layer_flops / s / 1e12 / tc_sus,
+             "tflops_frac_burst": layer_flops / s / 1e12 / tc_burst, "algorithmic_bytes": layer_bytes,
+             "algorithmic_flops": layer_flops,
+             "bound": "hbm" if layer_bytes / (peaks["hbm_gbs"] * 1e9) >= layer_flops / (tc_sus * 1e12) else "tensor"}
+    kern_bytes, kern_flops = kernel_bytes_flops(w, touched, fp8)
     dom = max(ktimes.items(), key=lambda kv: kv[1][1])[0] if ktimes else None
-    H, I, E, k = w.H, w.I, w.E, w.k
-    wb = 1 if args.fp8 else 2   # bytes per weight (e4m3 or bf16); e4m3 adds one fp32 scale per weight row
-    ab = 1 if args.fp8 else 2   # bytes per GEMM input activation
-    gate_up_bytes = (touched + 1) * 2 * I * (H * wb + (4 if args.fp8 else 0)) + (T * k + T) * H * ab + (T * k + T) * I * 2
-    down_bytes = (touched + 1) * H * (I * wb + (4 if args.fp8 else 0)) + (T * k + T) * I * ab + (T * k + T) * H * 2
-    kern_bytes = {"expert_gateup": gate_up_bytes, "expert_down": down_bytes}
-    kern_flops = {"expert_gateup": 2.0 * (T * k + T) * 2 * I * H, "expert_down": 2.0 * (T * k + T) * H * I}
     roof = None
     if dom in kern_bytes:
         launches, tot = ktimes[dom]
         avg_s = tot / launches / 1e3
-        intensity = kern_flops[dom] / kern_bytes[dom]
-        # the tensor peak of the contraction's own dtype: e4m3 = the measured bf16 peak x 2, the
-        # nominal dense ratio (4.5 / 2.25 PFLOP/s)
-        tc_peak = peaks["bf16_tflops_sustained"] * (2.0 if args.fp8 else 1.0)
-        tc_src = ("MEASURED_PEAKS.json bf16_tflops_sustained x 2 (nominal e4m3 / bf16 ratio)" if args.fp8
-                  else "MEASURED_PEAKS.json bf16_tflops_sustained")
-        ridge = tc_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
-        traffic = profiled_traffic(dom, w.name + ("_fp8" if args.fp8 else ""))
-        if intensity < ridge:
-            ach = kern_bytes[dom] / avg_s / 1e9
-            roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": ach / peaks["hbm_gbs"], "traffic": traffic,
-                    "algorithmic_bytes": kern_bytes[dom], "avg_launch_ms": avg_s * 1e3,
+        hbm_ach = kern_bytes[dom] / avg_s / 1e9
+        tc_ach = kern_flops[dom] / avg_s / 1e12
+        t_hbm = kern_bytes[dom] / (peaks["hbm_gbs"] * 1e9)
+        t_tc = kern_flops[dom] / (tc_sus * 1e12)
+        traffic = profiled_traffic(dom, w.name + ("_fp8" if fp8 else ""))
+        common = {"kernel": dom, "traffic": traffic, "algorithmic_bytes": kern_bytes[dom],
+                  "algorithmic_flops": kern_flops[dom], "avg_launch_ms": avg_s * 1e3,
+                  "hbm_gbs": hbm_ach, "hbm_frac": hbm_ach / peaks["hbm_gbs"], "tflops": tc_ach,
+                  "tflops_frac_sustained": tc_ach / tc_sus, "tflops_frac_burst": tc_ach / tc_burst}
+        tc_name = "bf16_tflops{}" + (" x 2 (nominal e4m3 / bf16 ratio)" if fp8 else "")
+        if t_hbm >= t_tc:
+            roof = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": hbm_ach / peaks["hbm_gbs"], **common,
                     "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_src})"}
         else:
-            ach = kern_flops[dom] / avg_s / 1e12
-            roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": tc_peak,
-                    "unit": "TFLOP/s", "frac": ach / tc_peak, "traffic": traffic, "algorithmic_flops": kern_flops[dom],
-                    "avg_launch_ms": avg_s * 1e3, "peak_source": f"{tc_src} ({peak_src})"}
-    layer_bytes = (touched + 1) * 3 * H * I * wb + E * H * 4 + 2 * T * H * 2
-    layer_flops = 2.0 * T * (k + 1) * 3 * H * I
+            roof = {"bound": "tensor", "achieved": tc_ach, "peak": tc_sus, "unit": "TFLOP/s",
+                    "frac": tc_ach / tc_sus, **common,
+                    "peak_source": f"MEASURED_PEAKS.json {tc_name.format('_sustained')} ({peak_src}); the burst "
+                                   f"peak {tc_burst:.1f} gives tflops_frac_burst"}
 
-    line = {"metric": METRIC, "value": world * T / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+    entry = {"value": world * T / s, "unit": UNIT, "ms_per_step": ms, "step_ms": spread,
+             "config": {**workload_config(w), **({"diag": True} if args.diag else {}),
+                        **({"experts": "e4m3, per-row fp32 scales; router fp32"} if fp8 else {})},
+             "layer": layer, "experts": experts,
+             "kernels_ms_per_step": {n: t / ksteps for n, (_, t) in sorted(ktimes.items(), key=lambda kv: -kv[1][1])},
+             "roofline": roof,
+             "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": T * H * 2,
+                     "d2h_bytes_per_step": T * H * 2, "ms_per_step": e2e_ms},
+             "gpu_launches": launches_per_step * args.steps, "launches_per_step": launches_per_step,
+             "clocks": clk.summary()}
+    del ws, x, out
+    return entry, gpu_idx
+
+
+def run_ours(args):
+    import torch
+
+    import sparse_moe_layer_smoe_b200 as smoe
+    import synth
+
+    rank, local, world = dist_env()
+    torch.cuda.set_device(local)
+    init_dist(world, "nccl")
+    dev = torch.device("cuda", local)
+    head = synth.WORKLOADS[args.workload]
+    extra = [] if args.workloads in ("", "none") else [n for n in args.workloads.split(",") if n != head.name]
+    for n in extra:
+        if synth.WORKLOADS[n].H != head.H or synth.WORKLOADS[n].E != head.E or synth.WORKLOADS[n].I != head.I:
+            raise SystemExit(f"--workloads: {n} has another layer shape than {head.name}")
+    cfg = smoe.config(head.H, head.E, head.k, head.I, head.Is, head.route_scale)
+
+    # the layer's weights, shared by every workload of this shape (same seed)
+    experts = synth.dev_experts(head, device=dev)
+    packed = smoe.pack_weights_fp8(cfg, *experts) if args.fp8 else smoe.pack_weights(cfg, *experts)
+    torch.cuda.synchronize()
+    del experts
+    torch.cuda.empty_cache()
+
+    results = {}
+    for name in [head.name] + extra:
+        results[name] = measure(smoe, synth.WORKLOADS[name], packed, args, dev, headline=(name == head.name))
+
+    entry, _ = results[head.name]
+    line = {"metric": METRIC, "value": entry["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": entry["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3" if args.fp8 else "bf16", "data": "synthetic",
-            "config": {**workload_config(w), **({"diag": True} if args.diag else {}),
-                       **({"experts": "e4m3, per-row fp32 scales; router fp32"} if args.fp8 else {})},
-            "layer": {"hbm_gbs": layer_bytes / (ms / 1e3) / 1e9, "tflops": layer_flops / (ms / 1e3) / 1e12,
-                      "experts_touched": touched, "algorithmic_bytes": layer_bytes},
-            "kernels_ms_per_step": {n: t / ksteps for n, (_, t) in sorted(ktimes.items(), key=lambda kv: -kv[1][1])},
-            "roofline": roof,
-            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": T * H * 2,
-                    "d2h_bytes_per_step": T * H * 2, "ms_per_step": e2e_ms},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk.summary()}
+            "config": entry["config"], "layer": entry["layer"], "experts": entry["experts"],
+            "step_ms": entry["step_ms"], "kernels_ms_per_step": entry["kernels_ms_per_step"],
+            "roofline": entry["roofline"], "e2e": entry["e2e"], "gpu_launches": entry["gpu_launches"],
+            "clocks": entry["clocks"],
+            "workloads": {n: {kk: vv for kk, vv in e.items() if kk != "config"} | {"T": synth.WORKLOADS[n].T}
+                          for n, (e, _) in results.items()}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, args.cpu_sample_tokens, args.cpu_seconds)
+        for n, (e, gidx) in results.items():
+            line["workloads"][n]["routing"] = routing_check(synth.WORKLOADS[n], gidx)
+        line["routing"] = line["workloads"][head.name]["routing"]
+        line["cpu_baseline"] = cpu_baseline(head, args.cpu_sample_tokens, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     import torch.distributed as dist

@@ -295,14 +295,19 @@ SMOE_API smoe_status_t smoe_timing_end(smoe_kernel_time_t* out, int32_t cap, int
  * inference runtime hands only its input and output buffers, or a serving path where
  * cudaMalloc is forbidden after start-up because it can synchronise the device and stall.
  * The pages have no counterpart to this entry point; it exists only for such callers.
- * Same arguments and results as smoe_route, without the workspace. Its scratch (the router's
- * K-split partial logits: splits x T x E x 4 bytes, 9.4 MB at T = 8192, E = 288) is a static
- * device array of SMOE_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until the
- * process exits; a T that needs more returns SMOE_ERR_WORKSPACE before any launch. The first
- * call on each device looks up the array's device address (cudaGetSymbolAddress, with that
- * device current); make that first call before any stream capture. Every call shares the one
- * array and keeps nothing from earlier calls: calls that overlap on the GPU (several streams or
- * host threads) race on it, so the caller must serialise them. Allocates and frees nothing. */
+ * Same arguments, checks and results as smoe_route, without the workspace; it always runs the
+ * CUDA-core router kernels. Its scratch (the router's K-split partial logits,
+ * splits x T x E x 4 bytes) is a static device array of SMOE_NOALLOC_SCRATCH_BYTES that every
+ * GPU loading the library holds until the process exits; a T that needs more returns
+ * SMOE_ERR_WORKSPACE before any launch. Large batches run with a K split of 1 (at E = 288 on
+ * a 148-SM B200: every batch above 3,136 tokens), so the largest batch is
+ * floor(16 MiB / (E x 4)) = 14,563 tokens at E = 288; smaller batches use up to 16 splits and
+ * fit too (at most 9.4 MB at E = 288). The array's device address is looked up
+ * (cudaGetSymbolAddress) on every call in the current context; the first call on each device
+ * or context also loads the library's device code there, so make that first call before any
+ * stream capture. Every call shares the one array and keeps nothing from earlier calls:
+ * calls that overlap on the GPU (several streams or host threads) race on it, so the caller
+ * must serialise them. Allocates and frees nothing. */
 #define SMOE_NOALLOC_SCRATCH_BYTES (16u << 20)
 SMOE_API smoe_status_t smoe_route_noalloc(const smoe_config_t* cfg, const smoe_bf16_t* x, int64_t T,
                                           const float* w_router, const float* bias, int32_t* topk_idx,

@@ -137,12 +137,15 @@ int32_t so_threads(void) { return thread_count(); }
 
 // bf16 bit patterns -> fp64, exactly: the bf16 bits are the upper half of an fp32.
 void so_bf16_to_f64(const uint16_t* in, int64_t n, double* out) {
-    for (int64_t i = 0; i < n; ++i) {
-        const uint32_t bits = static_cast<uint32_t>(in[i]) << 16;
-        float f;
-        std::memcpy(&f, &bits, sizeof f);
-        out[i] = static_cast<double>(f);
-    }
+    const int64_t block = 1 << 16;
+    parallel_for((n + block - 1) / block, [&](int64_t b) {
+        for (int64_t i = b * block; i < std::min(n, (b + 1) * block); ++i) {
+            const uint32_t bits = static_cast<uint32_t>(in[i]) << 16;
+            float f;
+            std::memcpy(&f, &bits, sizeof f);
+            out[i] = static_cast<double>(f);
+        }
+    });
 }
 
 // fp32 -> fp64, exactly.

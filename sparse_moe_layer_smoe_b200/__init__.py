@@ -20,6 +20,7 @@ STATUS = {0: "SMOE_OK", 1: "SMOE_ERR_INVALID_ARG", 2: "SMOE_ERR_UNSUPPORTED", 3:
           4: "SMOE_ERR_CUDA", 5: "SMOE_ERR_DEVICE", 6: "SMOE_ERR_TIMEOUT"}
 SMOE_OK, SMOE_ERR_INVALID_ARG, SMOE_ERR_UNSUPPORTED, SMOE_ERR_WORKSPACE = 0, 1, 2, 3
 SMOE_ERR_CUDA, SMOE_ERR_DEVICE, SMOE_ERR_TIMEOUT = 4, 5, 6
+SMOE_NOALLOC_SCRATCH_BYTES = 16 << 20   # include/stepmoe.h: the allocation-free router's static scratch
 
 
 class SmoeConfig(ctypes.Structure):

@@ -116,31 +116,7 @@ using namespace smoe;
 
 namespace {
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-smoe_status_t check_T(const smoe_config_t* c, int64_t T) {
-    if (T < 0) return SMOE_ERR_INVALID_ARG;
-    if (T > (int64_t)0x7FFFFFFF / (c->top_k + 1)) return SMOE_ERR_UNSUPPORTED;
-    return SMOE_OK;
-}
-
 smoe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? SMOE_OK : SMOE_ERR_CUDA; }
-
-#define SMOE_TRY(expr)                        \
-    do {                                      \
-        smoe_status_t _s = (expr);            \
-        if (_s != SMOE_OK) return _s;         \
-    } while (0)
-
-#define SMOE_REQUIRE_PTR(p)                                      \
-    do {                                                         \
-        if ((p) == nullptr || !aligned16(p)) return SMOE_ERR_INVALID_ARG; \
-    } while (0)
-
-#define SMOE_OPTIONAL_PTR(p)                                     \
-    do {                                                         \
-        if ((p) != nullptr && !aligned16(p)) return SMOE_ERR_INVALID_ARG; \
-    } while (0)
 
 smoe_status_t check_ws(const smoe_config_t* c, int64_t T, const void* ws, size_t ws_bytes, bool forward,
                        bool fp8 = false) {

@@ -16,6 +16,32 @@ constexpr int kPermuteTokensPerBlock = 256;
 
 inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
 
+// Argument checks shared by every entry point (host side, before any launch).
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// T: negative -> invalid; so large that the T*k + T rows overflow int32 -> unsupported.
+inline smoe_status_t check_T(const smoe_config_t* c, int64_t T) {
+    if (T < 0) return SMOE_ERR_INVALID_ARG;
+    if (T > (int64_t)0x7FFFFFFF / (c->top_k + 1)) return SMOE_ERR_UNSUPPORTED;
+    return SMOE_OK;
+}
+
+#define SMOE_TRY(expr)                        \
+    do {                                      \
+        smoe_status_t _s = (expr);            \
+        if (_s != SMOE_OK) return _s;         \
+    } while (0)
+
+#define SMOE_REQUIRE_PTR(p)                                                     \
+    do {                                                                        \
+        if ((p) == nullptr || !smoe::aligned16(p)) return SMOE_ERR_INVALID_ARG; \
+    } while (0)
+
+#define SMOE_OPTIONAL_PTR(p)                                                    \
+    do {                                                                        \
+        if ((p) != nullptr && !smoe::aligned16(p)) return SMOE_ERR_INVALID_ARG; \
+    } while (0)
+
 // Router plan for T tokens. CUDA cores: tokens per CTA, experts per CTA, K splits. Tensor cores
 // (tc, large T): W_r split into three bf16 pieces in the workspace, token tile nt.
 struct RouterPlan {

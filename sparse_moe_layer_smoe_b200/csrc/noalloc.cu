@@ -7,40 +7,18 @@
 // partial logits) lives in a file-scope device array of SMOE_NOALLOC_SCRATCH_BYTES, which every
 // GPU that loads the library holds until the process exits.
 //
-// In host code the array's name is only a host-side stand-in, never a device address, so its
-// device address is looked up here once per device with cudaGetSymbolAddress (the lookup runs
-// on the first call made with that device current) and passed to the kernels.
-#include <mutex>
-
+// In host code the array's name is only a host-side stand-in, never a device address. Its
+// device address belongs to the module instance loaded in the current context, so it is looked
+// up with cudaGetSymbolAddress on every call, with the caller's device current: a host that
+// runs its own (non-primary) contexts, or resets a device and so reloads the module, gets the
+// address that is valid now. The first call on each device (or context) is the one that loads
+// the module there; after that the lookup is a table read.
 #include "internal.h"
 
 namespace smoe {
 namespace {
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[SMOE_NOALLOC_SCRATCH_BYTES];
-
-constexpr int kMaxDev = 64;
-void* g_scratch_ptr[kMaxDev] = {nullptr};
-std::mutex g_scratch_mu;
-
-// Device address of the static scratch on the current device (looked up once per device).
-cudaError_t scratch_address(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
-    return cudaSuccess;
-}
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 }  // namespace smoe
@@ -50,22 +28,22 @@ using namespace smoe;
 extern "C" smoe_status_t smoe_route_noalloc(const smoe_config_t* c, const smoe_bf16_t* x, int64_t T,
                                             const float* w_router, const float* bias, int32_t* topk_idx,
                                             float* topk_w, float* logits_opt, void* stream) {
-    smoe_status_t st = smoe_check_config(c);
-    if (st != SMOE_OK) return st;
-    if (T < 0) return SMOE_ERR_INVALID_ARG;
-    if (T > (int64_t)0x7FFFFFFF / (c->top_k + 1)) return SMOE_ERR_UNSUPPORTED;
+    // the same argument checks as smoe_route, before any launch
+    SMOE_TRY(smoe_check_config(c));
+    SMOE_TRY(check_T(c, T));
     launches_reset();
     if (T == 0) return SMOE_OK;
-    const void* req[] = {x, w_router, bias, topk_idx, topk_w};
-    for (const void* p : req)
-        if (p == nullptr || !aligned16(p)) return SMOE_ERR_INVALID_ARG;
-    if (logits_opt != nullptr && !aligned16(logits_opt)) return SMOE_ERR_INVALID_ARG;
+    SMOE_REQUIRE_PTR(x);
+    SMOE_REQUIRE_PTR(w_router);
+    SMOE_REQUIRE_PTR(bias);
+    SMOE_REQUIRE_PTR(topk_idx);
+    SMOE_REQUIRE_PTR(topk_w);
+    SMOE_OPTIONAL_PTR(logits_opt);
     const int sms = num_sms_current_device();
     const RouterPlan rp = router_plan(*c, T, sms, /*allow_tc=*/false);
-    const size_t need = rp.scratch_bytes;
-    if (need > (size_t)SMOE_NOALLOC_SCRATCH_BYTES) return SMOE_ERR_WORKSPACE;
+    if (rp.scratch_bytes > (size_t)SMOE_NOALLOC_SCRATCH_BYTES) return SMOE_ERR_WORKSPACE;
     void* scratch = nullptr;
-    if (scratch_address(&scratch) != cudaSuccess) return SMOE_ERR_CUDA;
+    if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || scratch == nullptr) return SMOE_ERR_CUDA;
     // Every element of the partial-logit area the kernels read is written first in the same
     // call, so nothing needs clearing.
     const cudaError_t e = launch_route(*c, x, T, w_router, bias, topk_idx, topk_w, logits_opt,

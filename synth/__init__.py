@@ -243,6 +243,11 @@ WORKLOADS = {
                         description="8 experts top-2 over 8192 tokens: ~2048 rows per expert, weights reused from L2"),
     "prefill_e32": Workload("prefill_e32", 900, 4096, 32, 8, 1280, 1280,
                             description="prefill-shaped small case for counter captures: T=900, 32 experts top-8"),
+    # profiling case: the skewed batch's kernel shape (mean ~114 rows per expert, Zipf popularity
+    # with 16 dead experts, 1-row to multi-tile groups) on 72 experts, ~2.3 GB of weights
+    "skewed_e72": Workload("skewed_e72", 1024, 4096, 72, 8, 1280, 1280, bias="zipf",
+                           description="skewed-shaped small case for counter captures: T=1024, 72 experts top-8, "
+                                       "Zipf bias, 16 dead"),
 }
 ZIPF_DEAD = 16
 ZIPF_FIXTURE = os.path.join(REPO, "tests", "golden", "zipf_bias.json")

@@ -95,6 +95,14 @@ def bf16_tensor_to_f64(t) -> np.ndarray:
     return oracle.bf16_to_f64(t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16))
 
 
+def stratified_tokens(T: int, n: int, rng) -> list:
+    """n tokens spread over the whole batch: one random token in each of n equal slices."""
+    if T <= n:
+        return list(range(T))
+    edges = np.linspace(0, T, n + 1).astype(int)
+    return [int(rng.integers(a, b)) for a, b in zip(edges[:-1], edges[1:]) if b > a]
+
+
 def assert_close(gpu: np.ndarray, ref: np.ndarray, what: str, rel_fro=REL_FRO, rel_max=REL_MAX):
     err = gpu - ref
     fro = np.linalg.norm(err) / max(np.linalg.norm(ref), 1e-300)

@@ -148,3 +148,10 @@ def test_workspace_checks():
     fneed = smoe.smoe_workspace_bytes(c, 64)
     assert L.smoe_forward(cp, 16, 64, 16, 16, 16, 16, 256, fneed - 1, None) == smoe.SMOE_ERR_WORKSPACE
     assert L.smoe_combine(cp, 16, 16, 16, 4, 16, 256, 255, None) == smoe.SMOE_ERR_WORKSPACE
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    import re
+    text = open(smoe.HEADER).read()
+    m = re.search(r"#define SMOE_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
+    assert m and int(m.group(1)) << int(m.group(2)) == smoe.SMOE_NOALLOC_SCRATCH_BYTES

@@ -55,3 +55,4 @@ def test_reference_arm_prints_on_rank_0_only():
     line = json.loads(p.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["steps"] == 3 and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert "C++" in line["cpu_baseline"]["implementation"] and line["cpu_baseline"]["cores"] >= 1

@@ -7,10 +7,12 @@ seeded inputs, on all five workloads, at their full sizes.
   fp32 logits within an fp32 accumulation bound;
 * permute: counts, offsets, perm_row, row_token and x_perm bit-exact;
 * expert_ffn: fed the oracle's permutation, outputs vs fp64 SwiGLU experts (all rows for the
-  tiny layer, sampled rows of every kind at the Step shape);
+  tiny layer; at the Step shape rows from every (group, token tile), both halves of each tile
+  and every trimmed tail tile, the shared expert's tiles included);
 * combine: fed seeded bf16 rows and the oracle's weights, vs the fp64 formula within 1 bf16 ulp;
 * forward (the launch configuration bench.py times): the whole layer vs the oracle, dense-masked
-  for tiny and decode, sparse on sampled tokens (incl. near-tie and spike rows) otherwise; and a
+  for tiny and decode, sparse on >= 256 tokens spread over the batch (plus near-tie and spike
+  rows) otherwise; and a
   degenerate routing collapse (every token to the same 8 experts) on both GEMM kernels.
 """
 import numpy as np
@@ -19,7 +21,7 @@ import pytest
 import oracle
 import synth
 from layer_fixtures import (ALL_WORKLOADS, HostExperts, assert_close, bf16_tensor_to_f64, cfg_of, device_inputs,
-                            host_route, host_x64, limit_of, selection_ok)
+                            host_route, host_x64, limit_of, selection_ok, stratified_tokens)
 
 pytestmark = pytest.mark.gpu
 
@@ -69,7 +71,7 @@ def test_route_parity(name):
     scale = np.abs(host_x64(name)).max(axis=1, keepdims=True) * 0.1 + 1.0
     assert np.all(np.abs(gl - r.logits) <= 2e-4 * scale), np.abs(gl - r.logits).max()
 
-    near = 0
+    near = swapped = 0
     for t in range(T):
         gset = tuple(sorted(gi[t].tolist()))
         assert len(set(gset)) == w.k and min(gset) >= 0 and max(gset) < w.E
@@ -80,6 +82,7 @@ def test_route_parity(name):
         # order: descending oracle biased score, up to inner ties closer than the tie tolerance
         b = r.bhat[t, gi[t]]
         assert np.all(b[:-1] >= b[1:] - oracle.NEAR_TIE_EPS), f"token {t}: order {gi[t]} vs {r.idx[t]}"
+        swapped += int(gset == tuple(sorted(r.idx[t].tolist())) and not np.array_equal(gi[t], r.idx[t]))
         if not r.near_tie[t]:
             # weights matched by expert id: the oracle's weight of each selected expert
             ref_w = dict(zip(r.idx[t].tolist(), r.w[t].tolist()))
@@ -88,7 +91,8 @@ def test_route_parity(name):
             s_sel = r.s[t, gi[t]]
             assert np.allclose(gw[t], oracle.normalise(s_sel, w.route_scale), rtol=1e-5, atol=0)
     assert np.allclose(gw.sum(axis=1), w.route_scale, rtol=1e-6)
-    print(f"{name}: {near} near-tie tokens of {T}")
+    print(f"{name}: {near} near-tie tokens of {T}; {swapped} tokens with the oracle's set in another order "
+          f"(every swap within the 1e-5 band)")
 
 
 @pytest.mark.parametrize("T", [37, 700, 2100])   # the small-batch, mid-batch and tensor-core router plans
@@ -149,18 +153,33 @@ def test_permute_parity(name):
 
 
 # ------------------------------------------------------------------------------ expert FFN
-def _ffn_sample_rows(offsets, T, k, n_groups=6):
-    """Rows to check: first/last row of a spread of routed groups, random routed rows, shared rows."""
+def _token_tile_rows(offsets, T, k, rng):
+    """Rows of y that reach every (group, token tile) of the expert GEMMs: in each tile its first
+    and last rows, the first row of its second half and one random row of each half (a CTA pair
+    holds one half of a tile in each CTA), so every trimmed tail tile and the shared expert's
+    tiles are checked too. The tiling restates the kernels' documented rule: the launch's largest
+    tile is the smallest power of two >= 1.25 x the mean rows per routed expert (16..256), and a
+    group of r rows uses the smallest power of two >= r, clamped to [16, that largest tile]."""
     E = len(offsets) - 1
-    nonempty = [e for e in range(E) if offsets[e + 1] > offsets[e]]
-    pick = sorted(set(np.linspace(0, len(nonempty) - 1, n_groups).astype(int).tolist()))
-    rows = []
-    for i in pick:
-        e = nonempty[i]
-        rows += [offsets[e], offsets[e + 1] - 1]
-    rows += RNG.integers(0, T * k, 8).tolist()
-    rows += [T * k, T * k + T - 1] + (T * k + RNG.integers(0, T, 4)).tolist()
-    return sorted(set(int(v) for v in rows))
+    nt_max = 16
+    while nt_max < 256 and nt_max < 1.25 * T * k / E:
+        nt_max *= 2
+    groups = [(int(offsets[e]), int(offsets[e + 1])) for e in range(E)] + [(T * k, T * k + T)]
+    rows = set()
+    tiles = 0
+    for a, b in groups:
+        if b == a:
+            continue
+        nt = 16
+        while nt < b - a and nt < nt_max:
+            nt *= 2
+        for s in range(a, b, nt):
+            end, half = min(s + nt, b), s + nt // 2
+            rows |= {s, end - 1, int(rng.integers(s, min(half, end)))}
+            if half < end:
+                rows |= {half, int(rng.integers(half, end))}
+            tiles += 1
+    return sorted(rows), tiles
 
 
 @pytest.mark.parametrize("mode", ["gather", "x_perm"])
@@ -186,7 +205,13 @@ def test_expert_ffn_parity(name, mode):
     x64 = host_x64(name)
     experts = HostExperts(w)
     group_of = np.searchsorted(offsets, np.arange(T * k), side="right") - 1
-    rows = list(range(T * k + T)) if name == "tiny" else _ffn_sample_rows(offsets, T, k)
+    if name == "tiny":
+        rows, tiles = list(range(T * k + T)), None
+    else:
+        rows, tiles = _token_tile_rows(offsets, T, k, RNG)
+    if w.bias == "zipf":   # the dead experts own no rows
+        dead = np.nonzero(synth.zipf_ranks(w) > w.E - synth.ZIPF_DEAD)[0]
+        assert len(dead) == synth.ZIPF_DEAD and np.all(offsets[dead + 1] == offsets[dead])
     spikes = synth.spike_rows(w)
     if len(spikes):   # rows of the x50 spike tokens: routed ones and their shared rows
         rows = sorted(set(rows) | set(np.nonzero(np.isin(row_token, spikes))[0][:6].tolist())
@@ -208,7 +233,7 @@ def test_expert_ffn_parity(name, mode):
     assert np.all(np.isfinite(gy[rows]))
     fro, mx = assert_close(gy[rows], ref, f"{name} expert_ffn ({mode})")
     assert torch.isfinite(y.float()).all()   # every row written
-    print(f"{name}: expert_ffn ({mode}) rows={len(rows)} rel_fro={fro:.2e} rel_max={mx:.2e}")
+    print(f"{name}: expert_ffn ({mode}) rows={len(rows)} token tiles={tiles} rel_fro={fro:.2e} rel_max={mx:.2e}")
 
 
 # ------------------------------------------------------------------------------ combine
@@ -292,7 +317,7 @@ def test_forward_parity_sampled(name):
     wt = torch.empty(w.T, w.k, dtype=torch.float32, device="cuda")
     smoe.smoe_route(cfg, x, w.T, wr, bias, idx, wt, None, _ws(cfg, w.T))
     r = host_route(name)
-    rows = {0, w.T - 1, *RNG.integers(0, w.T, 6).tolist()}
+    rows = {0, w.T - 1, *stratified_tokens(w.T, 256, RNG)}
     rows |= set(np.nonzero(r.near_tie)[0][:3].tolist())
     rows |= set(synth.spike_rows(w).tolist())
     rows = sorted(rows)
