@@ -88,8 +88,13 @@ WsLayout ws_layout(const smoe_config_t& c, int64_t T, int num_sms) {
     L.offsets = o;   o += align_up((size_t)(E + 1) * 4);
     L.perm_row = o;  o += align_up((size_t)routed * 4);
     L.row_token = o; o += align_up((size_t)routed * 4);
+    // small token tiles: smoe_forward's gate/up GEMM writes the shared expert's rows of h while
+    // the routing may still use the scratch union, so its h lies outside the union
+    const bool small_tiles = choose_token_tile(c, T) <= kGatherMaxTile;
+    L.ffn_h_fwd = small_tiles ? o : L.ffn_h;
+    if (small_tiles) o += h_b;
     L.x_perm = o;    // only when smoe_forward materialises the permuted rows (large token tiles)
-    if (choose_token_tile(c, T) > kGatherMaxTile) o += align_up((size_t)routed * H * 2);
+    if (!small_tiles) o += align_up((size_t)routed * H * 2);
     L.y = o;         o += align_up((size_t)(routed + T) * H * 2);
     L.row_norm = o;  o += align_up((size_t)routed * 4);
     L.total = o;
@@ -316,6 +321,11 @@ smoe_status_t smoe_combine(const smoe_config_t* c, const smoe_bf16_t* y, const i
 
 namespace {
 
+#ifndef SMOE_SHARED_PREWAIT
+#define SMOE_SHARED_PREWAIT 1
+#endif
+constexpr bool kSharedPrewait = SMOE_SHARED_PREWAIT != 0;
+
 smoe_status_t forward_impl(const smoe_config_t* c, const smoe_bf16_t* x, int64_t T, const float* w_router,
                            const float* bias, const void* packed, smoe_bf16_t* out, const smoe_diag_t* diag, void* ws,
                            size_t ws_bytes, void* stream, bool fp8 = false) {
@@ -358,12 +368,19 @@ smoe_status_t forward_impl(const smoe_config_t* c, const smoe_bf16_t* x, int64_t
     const bool gather = choose_token_tile(*c, T) <= kGatherMaxTile;
     uint16_t* x_perm = gather ? nullptr : at<uint16_t>(ws, L.x_perm);
     if (!fp8) {
+        // Small token tiles: the shared expert's gate/up units run in the GEMM before its
+        // dependency wait, overlapping the routing. Their inputs are x (this call's input,
+        // complete before the router's first kernel passed its own wait) and the packed weights;
+        // their output rows of h lie outside the scratch the routing uses. The one-CTA
+        // permutation lets the GEMM launch at once to make room for that.
+        const bool prewait = gather && kSharedPrewait && shared_prewait_fits(*c, T, sms);
         if (e == cudaSuccess)
             e = launch_permute(*c, idx, T, gather ? nullptr : x, at<int32_t>(ws, L.counts), offsets, perm_row,
-                               row_token, x_perm, at<int32_t>(ws, L.perm_hist), at<int32_t>(ws, L.perm_base), err, s);
+                               row_token, x_perm, at<int32_t>(ws, L.perm_hist), at<int32_t>(ws, L.perm_base), err, s,
+                               0, prewait);
         if (e == cudaSuccess)
-            e = launch_expert_ffn(*c, x, x_perm, row_token, offsets, T, packed, y, at<uint16_t>(ws, L.ffn_h), err, sms,
-                                  s);
+            e = launch_expert_ffn(*c, x, x_perm, row_token, offsets, T, packed, y, at<uint16_t>(ws, L.ffn_h_fwd), err,
+                                  sms, s, prewait);
     } else {
         // e4m3: x was quantised per token by the top-k kernel; the permuted copy (large tiles) is
         // of the e4m3 rows, moved by the same gather kernel as 2-byte pairs

@@ -91,6 +91,9 @@ struct GemmParams {
     const float* act_scale;   // per token (gate/up) or per activation row (down)
     const int32_t* scale_tok; // gate/up: routed activation row -> token (act_scale index); down: nullptr
     int scale_shared_base;    // act_scale index of the shared group's first row (0, or T*k for down)
+    int shared_first = 0;     // list the shared group's tiles before the routed groups' (else after)
+    int shared_prewait = 0;   // single-CTA kernel: the shared group's units run before the dependency
+                              // wait (its inputs must not come from the kernels just before this one)
 };
 
 // What a launch computes: the down projection, the fused gate/up + SiLU*mul, or router logits.
@@ -120,7 +123,7 @@ __host__ __device__ inline int max_token_tiles(int E, int routed_rows, int T, in
 __host__ __device__ inline size_t gemm_smem_bytes(int stages, int stage_b, int E, int max_tiles) {
     size_t b = 1024;                                       // alignment slack
     b += (size_t)stages * stage_b;
-    b += sizeof(uint64_t) * (2 * (size_t)stages + 5);      // full, empty, tfull[2], tempty[2], drain
+    b += sizeof(uint64_t) * (2 * (size_t)stages + 6);      // full, empty, tfull[2], tempty[2], drain, tab_ready
     b += 16;                                               // tmem slot, abort flag, tile count
     b += sizeof(int32_t) * ((size_t)max_tiles + E + 1);    // tiles[max_tiles], offs[E+1]
     return b;
@@ -192,11 +195,15 @@ __device__ __forceinline__ int snake_unit(int i, int w, int W, int total) {
 }
 
 // One warp: validate the offsets into offs[] (corrupt offsets: no routed work, the error word
-// set), then list the token tiles in tiles[] (entry g << 20 | nb) in group order. Returns the
-// tile count. Lane l owns a contiguous range of groups and one warp scan places its tiles:
-// every CTA of the launch builds the same table.
+// set), then list the token tiles in tiles[] (entry g << 20 | nb) in group order, the shared
+// group (g = E) last or first (shared_place); the shared group's first sh_skip
+// tiles are left out (they were computed before the table existed). Returns the tile count.
+// Lane l owns a contiguous range of groups and one warp scan places its tiles: every CTA of the
+// launch builds the same table.
+enum SharedPlace { kSharedLast = 0, kSharedFirst = 1 };
+
 __device__ int build_tile_table(const int32_t* offsets, int E, int T, int routed_rows, int nt_max, int max_tiles,
-                                int32_t* offs, int32_t* tiles, int32_t* err) {
+                                int32_t* offs, int32_t* tiles, int32_t* err, int shared_place, int sh_skip = 0) {
     const int lane = threadIdx.x & 31;
     bool bad = false;
     for (int i = lane; i <= E; i += 32) {
@@ -214,14 +221,16 @@ __device__ int build_tile_table(const int32_t* offsets, int E, int T, int routed
     __syncwarp();
     const int ngroups = E + 1;
     const int chunk = (ngroups + 31) / 32;
-    const int g0 = min(lane * chunk, ngroups), g1 = min(g0 + chunk, ngroups);
+    const int o0 = min(lane * chunk, ngroups), o1 = min(o0 + chunk, ngroups);
+    auto group_at = [&](int o) { return shared_place == kSharedFirst ? (o == 0 ? E : o - 1) : o; };   // position -> group
+    auto skip_of = [&](int g) { return g == E ? sh_skip : 0; };
     auto tiles_of = [&](int g) {
         const int rows = group_rows(g, E, T, offs);
         const int nt = group_tile(rows, nt_max);
-        return (rows + nt - 1) / nt;
+        return max((rows + nt - 1) / nt - skip_of(g), 0);
     };
     int local = 0;
-    for (int g = g0; g < g1; ++g) local += tiles_of(g);
+    for (int o = o0; o < o1; ++o) local += tiles_of(group_at(o));
     int incl = local;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -229,10 +238,11 @@ __device__ int build_tile_table(const int32_t* offsets, int E, int T, int routed
         if (lane >= off) incl += n;
     }
     int pos = incl - local;
-    for (int g = g0; g < g1; ++g) {
+    for (int o = o0; o < o1; ++o) {
+        const int g = group_at(o);
         const int nblk = tiles_of(g);
         for (int nb = 0; nb < nblk; ++nb, ++pos)
-            if (pos < max_tiles) tiles[pos] = (g << 20) | nb;
+            if (pos < max_tiles) tiles[pos] = (g << 20) | (nb + skip_of(g));
     }
     int n = __shfl_sync(0xFFFFFFFFu, incl, 31);
     if (n > max_tiles) {   // cannot happen for validated offsets; never read past the table
@@ -347,20 +357,33 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     uint64_t* tfull = empty + S;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* tab_ready = drain + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tab_ready + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* ntiles_slot = reinterpret_cast<int*>(tmem_slot + 2);
     int32_t* ttab = reinterpret_cast<int32_t*>(tmem_slot + 4);     // token tiles [max_tiles]
     int32_t* offs = ttab + p.max_tiles;                              // [E+1]
 
-    pdl_wait();
-    pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
     const int MB = p.n_out / 128;
     constexpr int EK = F8 ? 128 : BK;     // K elements per stage (128-byte rows either way)
     constexpr int TK = F8 ? 128 : 64;     // K elements per packed weight tile
     const int KB = p.K / EK / p.ksplit;   // k-blocks of one unit
+    const int upt = MB * p.ksplit;        // units per token tile
+    const int W = gridDim.x;
+
+    // Shared units before the dependency wait (shared_prewait): the shared group's rows are the
+    // rows of x and its weights are fixed, so its units need nothing the earlier kernels of this
+    // layer compute. As many whole shared tiles as one round of CTAs holds (one unit per CTA)
+    // run first, CTA b taking unit b; the table built once the offsets are known lists the
+    // shared group's other tiles first, then the routed ones, dealt over all CTAs.
+    const bool prewait = p.shared_prewait != 0 && p.row_token != nullptr;   // gather mode: a full producer warp
+    const int nt_sh = group_tile(p.T, p.nt_max);
+    const int pre_tiles = prewait ? min((p.T + nt_sh - 1) / nt_sh, W / upt) : 0;
+    const int n_shared = pre_tiles * upt;   // <= W
+    auto shared_unit = [&](int) { const int s = blockIdx.x; return Unit{E, s % upt, s / upt, nt_sh}; };
+    auto n_shared_mine = [&]() { return blockIdx.x < (unsigned)n_shared ? 1 : 0; };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -372,6 +395,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             mbar_init(smem_u32(&tempty[a]), 128);
         }
         mbar_init(smem_u32(drain), 1);
+        mbar_init(smem_u32(tab_ready), 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -387,16 +411,35 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 tma_prefetch_desc(&maps.sh[i]);
             }
     }
-    if (warp == 2) {
-        const int n = build_tile_table(p.offsets, E, p.T, p.routed_rows, p.nt_max, p.max_tiles, offs, ttab, p.err);
-        if (lane == 0) *ntiles_slot = n;
+    // The set-up above reads nothing an earlier kernel writes, so it overlaps that kernel's tail
+    // (this CTA's shared memory rules out sharing an SM, hence TMEM, with another GEMM CTA).
+    if (!prewait) {
+        // everything below may read the earlier kernels' results: wait for them, then list the
+        // token tiles
+        pdl_wait();
+        pdl_launch_dependents();
+        if (warp == 2) {
+            const int n = build_tile_table(p.offsets, E, p.T, p.routed_rows, p.nt_max, p.max_tiles, offs, ttab,
+                                           p.err, p.shared_first != 0 ? kSharedFirst : kSharedLast);
+            if (lane == 0) *ntiles_slot = n;
+        }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int upt = MB * p.ksplit;   // units per token tile
-    const int total = *ntiles_slot * upt;
+
+    // Before its first routed unit each role waits for the tile table: built above (plain
+    // launch), or by the producer warp once the offsets are there (shared_prewait), which then
+    // arrives on tab_ready. Returns the routed unit count.
+    auto await_table = [&]() -> int {
+        if (prewait) {
+            if (!mbar_wait(smem_u32(tab_ready), 0u, p.err, abort_flag, true)) return 0;
+            pdl_wait();
+            pdl_launch_dependents();
+        }
+        return *ntiles_slot * upt;
+    };
 
     // gather mode (row_token set) uses all 32 producer lanes; otherwise lane 0 alone, so the
     // stage refill path carries no warp-wide synchronisation
@@ -412,10 +455,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         int stage = 0;
         uint32_t phase = 0, armed = 0, armed_par = 0;
         bool ok = true;
-        for (int i = 0; ok && i * (int)gridDim.x < total; ++i) {
-            const int u = snake_unit(i, blockIdx.x, gridDim.x, total);
-            if (u < 0) continue;
-            Unit w = decode_unit(u, upt, ttab, offs, E, p.T, p.nt_max);
+        auto load_unit = [&](Unit w) {
             const int kb0 = (w.mb / MB) * KB;   // first k-block of this unit's K range
             w.mb %= MB;
             const int a_row = DUAL ? (w.g * MB + w.mb) * 256 : w.g * p.n_out + w.mb * 128;   // router: row-major
@@ -472,6 +512,25 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                 if (++stage == S) { stage = 0; phase ^= 1u; }
             }
+        };
+        for (int j = 0; ok && j < n_shared_mine(); ++j) load_unit(shared_unit(j));
+        if (prewait) {
+            // the offsets are final once the earlier kernels are done: list the routed tiles
+            pdl_wait();
+            pdl_launch_dependents();
+            const int n = build_tile_table(p.offsets, E, p.T, p.routed_rows, p.nt_max, p.max_tiles, offs, ttab, p.err,
+                                           kSharedFirst, pre_tiles);
+            if (lane == 0) {
+                *ntiles_slot = n;
+                mbar_arrive(smem_u32(tab_ready));
+            }
+            __syncwarp();
+        }
+        const int total = *ntiles_slot * upt;
+        for (int i = 0; ok && i * W < total; ++i) {
+            const int u = snake_unit(i, blockIdx.x, W, total);
+            if (u < 0) continue;
+            load_unit(decode_unit(u, upt, ttab, offs, E, p.T, p.nt_max));
         }
         // every load issued must land before the CTA may exit
         if (lane == 0)
@@ -484,13 +543,10 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         int stage = 0, acc = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
-        for (int i = 0; ok && i * (int)gridDim.x < total; ++i) {
-            const int u = snake_unit(i, blockIdx.x, gridDim.x, total);
-            if (u < 0) continue;
-            const Unit w = decode_unit(u, upt, ttab, offs, E, p.T, p.nt_max);
+        auto mma_unit = [&](const Unit& w) {
             const int n_mma = mma_cols(group_rows(w.g, E, p.T, offs) - w.nb * w.nt, w.nt);
             const uint32_t idesc = idesc0 | ((uint32_t)(n_mma >> 3) << 17);
-            if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, p.err, abort_flag, true)) break;
+            if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, p.err, abort_flag, true)) { ok = false; return; }
             tc_fence_after();
             const uint32_t d = tmem_base + (uint32_t)(acc * ACC_COLS);
             for (int kb = 0; kb < KB; ++kb) {
@@ -515,7 +571,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 umma_commit(smem_u32(&empty[stage]));
                 if (++stage == S) { stage = 0; phase ^= 1u; }
             }
-            if (!ok) break;
+            if (!ok) return;
             umma_commit(smem_u32(&tfull[acc]));
             if (NACC == 2) {
                 acc ^= 1;
@@ -523,6 +579,13 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             } else {
                 acc_phase ^= 1u;
             }
+        };
+        for (int j = 0; ok && j < n_shared_mine(); ++j) mma_unit(shared_unit(j));
+        const int total = ok ? await_table() : 0;
+        for (int i = 0; ok && i * W < total; ++i) {
+            const int u = snake_unit(i, blockIdx.x, W, total);
+            if (u < 0) continue;
+            mma_unit(decode_unit(u, upt, ttab, offs, E, p.T, p.nt_max));
         }
         // all MMAs issued by this thread must finish before TMEM is released
         umma_commit(smem_u32(drain));
@@ -533,10 +596,8 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         const int row = q * 32 + lane;     // accumulator row = output feature within the block
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int i = 0; i * (int)gridDim.x < total; ++i) {
-            const int u = snake_unit(i, blockIdx.x, gridDim.x, total);
-            if (u < 0) continue;
-            Unit w = decode_unit(u, upt, ttab, offs, E, p.T, p.nt_max);
+        bool ok = true;
+        auto epi_unit = [&](Unit w) {
             const int kp = w.mb / MB;   // K range of this unit (partial output kp)
             w.mb %= MB;
             const int rows = group_rows(w.g, E, p.T, offs);
@@ -544,7 +605,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             const int nvalid = min(w.nt, rows - w.nb * w.nt);
             float cs[8];
             if (F8) load_col_scales(p, w, nvalid, offs, lane, cs);
-            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.err, abort_flag, true)) break;
+            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.err, abort_flag, true)) { ok = false; return; }
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
             const int f = w.mb * 128 + row;
@@ -581,7 +642,18 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             } else {
                 acc_phase ^= 1u;
             }
+        };
+        for (int j = 0; ok && j < n_shared_mine(); ++j) epi_unit(shared_unit(j));
+        const int total = ok ? await_table() : 0;
+        for (int i = 0; ok && i * W < total; ++i) {
+            const int u = snake_unit(i, blockIdx.x, W, total);
+            if (u < 0) continue;
+            epi_unit(decode_unit(u, upt, ttab, offs, E, p.T, p.nt_max));
         }
+    }
+    if (prewait && warp == 1 && lane != 0) {   // the idle lanes of the MMA warp take part in the wait too
+        pdl_wait();
+        pdl_launch_dependents();
     }
 
     tc_fence_before();
@@ -631,8 +703,6 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
     int32_t* ttab = reinterpret_cast<int32_t*>(tmem_slot + 4);     // token tiles [max_tiles]
     int32_t* offs = ttab + p.max_tiles;                              // [E+1]
 
-    pdl_wait();
-    pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
@@ -668,8 +738,14 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
                 tma_prefetch_desc(&maps.sh[i]);
             }
     }
+    // The set-up above reads nothing an earlier kernel writes, so it overlaps that kernel's tail
+    // (this CTA's shared memory rules out sharing an SM, hence TMEM, with another GEMM CTA);
+    // everything below may read its results.
+    pdl_wait();
+    pdl_launch_dependents();
     if (warp == 2) {
-        const int n = build_tile_table(p.offsets, E, p.T, p.routed_rows, p.nt_max, p.max_tiles, offs, ttab, p.err);
+        const int n = build_tile_table(p.offsets, E, p.T, p.routed_rows, p.nt_max, p.max_tiles, offs, ttab, p.err,
+                                         p.shared_first != 0 ? kSharedFirst : kSharedLast);
         if (lane == 0) *ntiles_slot = n;
     }
     tc_fence_before();
@@ -982,6 +1058,10 @@ cudaError_t run_gemm_pair(const GemmMaps& maps, GemmParams p, int num_sms, cudaS
 
 }  // namespace
 
+#ifndef SMOE_SHARED_FIRST
+#define SMOE_SHARED_FIRST 1   // small-tile gate/up launches list the shared expert's tiles first
+#endif
+
 // Largest token tile of a launch: the smallest power of two >= 1.25 x the mean rows per routed
 // expert, 16..256. Groups with fewer rows use smaller tiles inside the kernel.
 #ifndef SMOE_TILE_FACTOR
@@ -994,6 +1074,16 @@ int choose_token_tile(const smoe_config_t& c, int64_t T) {
     return nt;
 }
 
+// Shared units before the wait only when all of them fit in one round of CTAs (decode-sized
+// batches): with more (the MTP batch's 16 tiles), the GEMM launched early competes with the
+// top-k kernel's CTAs for the SMs and the routing takes longer than the overlap saves.
+bool shared_prewait_fits(const smoe_config_t& c, int64_t T, int num_sms) {
+    const int nt = choose_token_tile(c, T);
+    int nt_sh = 16;
+    while (nt_sh < T && nt_sh < nt) nt_sh *= 2;
+    return (T + nt_sh - 1) / nt_sh * (c.inter / 128) <= num_sms;
+}
+
 size_t packed_gateup_bytes(const smoe_config_t& c) {
     return (size_t)(c.n_experts + 1) * 2 * c.inter * c.hidden * 2;
 }
@@ -1001,7 +1091,8 @@ size_t packed_down_bytes(const smoe_config_t& c) { return (size_t)(c.n_experts +
 
 cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const uint16_t* x_perm,
                               const int32_t* row_token, const int32_t* offsets, int64_t T, const void* packed,
-                              uint16_t* y, uint16_t* h, int32_t* err, int num_sms, cudaStream_t s) {
+                              uint16_t* y, uint16_t* h, int32_t* err, int num_sms, cudaStream_t s,
+                              bool shared_prewait) {
     constexpr int BK = SMOE_GEMM_BK;
     const int E = c.n_experts, H = c.hidden, I = c.inter, k = c.top_k;
     const int64_t routed = T * k;
@@ -1029,6 +1120,8 @@ cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const u
 
     GemmParams p1{offsets, E, (int)T, (int)routed, H, I, 0, (int)routed, nt, 0, 0, I, I, gather ? row_token : nullptr,
                   c.swiglu_limit, c.swiglu_limit_shared, 1, 0, h, nullptr, err};
+    p1.shared_first = gather && SMOE_SHARED_FIRST ? 1 : 0;
+    p1.shared_prewait = gather && !pairs && shared_prewait && shared_prewait_fits(c, T, num_sms) ? 1 : 0;
     cudaError_t e = pairs ? run_gemm_pair<MODE_GATEUP>(m1, p1, num_sms, s) : run_gemm<MODE_GATEUP>(m1, p1, num_sms, s);
     if (e != cudaSuccess) return e;
     GemmParams p2{offsets, E, (int)T, (int)routed, I, H, (int)routed, (int)routed, nt, 0, 0, H, H, nullptr, 0.f, 0.f, 1,
@@ -1073,6 +1166,7 @@ cudaError_t launch_expert_ffn_fp8(const smoe_config_t& c, const uint8_t* x_q, co
     p1.act_scale = s_x;
     p1.scale_tok = row_token;
     p1.scale_shared_base = 0;
+    p1.shared_first = gather && SMOE_SHARED_FIRST ? 1 : 0;
     cudaError_t e = pairs ? run_gemm_pair<MODE_GATEUP, true>(m1, p1, num_sms, s)
                           : run_gemm<MODE_GATEUP, true>(m1, p1, num_sms, s);
     if (e != cudaSuccess) return e;

@@ -61,6 +61,7 @@ struct WsLayout {
     size_t perm_hist = 0;        // [nblk][E] int32      (inside the union)
     size_t perm_base = 0;        // [nblk][E] int32      (inside the union)
     size_t ffn_h = 0;            // [T*k + T][I] bf16    (inside the union)
+    size_t ffn_h_fwd = 0;        // h of smoe_forward: outside the union for small token tiles
     size_t scratch_end = 0;
     size_t topk_idx = 0, topk_w = 0, counts = 0, offsets = 0, perm_row = 0, row_token = 0, x_perm = 0, y = 0;
     size_t row_norm = 0;         // [T*k] fp32 (smoe_forward_diag)
@@ -120,13 +121,19 @@ cudaError_t launch_route(const smoe_config_t& c, const uint16_t* x, int64_t T, c
 cudaError_t launch_router_gemm(const uint16_t* x, int64_t T, int H, const uint16_t* w_split, int e_pad, int E,
                                float* logits, int nt, int ksplit, int num_sms, cudaStream_t s);
 
+// early_trigger: the one-CTA permutation lets the next kernel launch before its own dependency
+// wait (that kernel then overlaps the routing; it still waits for this one's results).
 cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int64_t T, const uint16_t* x,
                            int32_t* counts, int32_t* offsets, int32_t* perm_row, int32_t* row_token,
                            uint16_t* x_perm, int32_t* hist, int32_t* base, int32_t* err, cudaStream_t s,
-                           int gather_cols = 0);   // row width in 2-byte units for the x_perm gather (0: hidden)
+                           int gather_cols = 0,   // row width in 2-byte units for the x_perm gather (0: hidden)
+                           bool early_trigger = false);
 
 // Largest token tile of an expert-GEMM launch for T tokens (16..256).
 int choose_token_tile(const smoe_config_t& c, int64_t T);
+
+// Whether smoe_forward runs the shared expert's gate/up units before the GEMM's dependency wait.
+bool shared_prewait_fits(const smoe_config_t& c, int64_t T, int num_sms);
 
 // smoe_forward reads routed rows straight from x (TMA row gathers) when the largest token tile
 // is at most this; above it, per-row gathers cost more than one gather kernel plus tile loads.
@@ -137,9 +144,13 @@ constexpr int kGatherMaxTile = SMOE_GATHER_MAX_TILE;
 
 // x_perm == nullptr selects gather mode: routed rows are read from x through row_token.
 // Returns cudaErrorNotSupported when the driver entry point for tensor maps is unavailable.
+// shared_prewait (gather mode): the gate/up kernel computes the shared expert's units before its
+// dependency wait, so x must not come from the two kernels launched just before it; h must
+// not overlap memory those kernels use.
 cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const uint16_t* x_perm,
                               const int32_t* row_token, const int32_t* offsets, int64_t T, const void* packed,
-                              uint16_t* y, uint16_t* h, int32_t* err, int num_sms, cudaStream_t s);
+                              uint16_t* y, uint16_t* h, int32_t* err, int num_sms, cudaStream_t s,
+                              bool shared_prewait = false);
 
 // row_norm_opt: when set, also ||y[r]||_2 of every routed row r (fp32, [T*k]).
 cudaError_t launch_combine(const smoe_config_t& c, const uint16_t* y, const int32_t* perm_row, const float* topk_w,

@@ -158,9 +158,12 @@ __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(const int3
                                                                       int E, int32_t* __restrict__ counts,
                                                                       int32_t* __restrict__ offsets,
                                                                       int32_t* __restrict__ perm_row,
-                                                                      int32_t* __restrict__ row_token, int32_t* err) {
+                                                                      int32_t* __restrict__ row_token, int32_t* err,
+                                                                      int early_trigger) {
+    // early_trigger: the next kernel may launch at once (its own wait still covers this one)
+    if (early_trigger) pdl_launch_dependents();
     pdl_wait();
-    pdl_launch_dependents();
+    if (!early_trigger) pdl_launch_dependents();
     extern __shared__ uint32_t smem[];
     uint32_t* wmask = smem;                                                  // [warps][E]
     int32_t* wbase = reinterpret_cast<int32_t*>(smem + kSmallWarps * E);     // [warps][E]
@@ -263,7 +266,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int64_t T, const uint16_t* x,
                            int32_t* counts, int32_t* offsets, int32_t* perm_row, int32_t* row_token,
                            uint16_t* x_perm, int32_t* hist, int32_t* base, int32_t* err, cudaStream_t s,
-                           int gather_cols) {
+                           int gather_cols, bool early_trigger) {
     const int E = c.n_experts, k = c.top_k;
     const int nblk = (int)((T + TB - 1) / TB);
     cudaError_t e;
@@ -277,7 +280,7 @@ cudaError_t launch_permute(const smoe_config_t& c, const int32_t* topk_idx, int6
         {
             LaunchTimer lt(K_PERMUTE_SCATTER, s);
             e = launch_pdl(permute_small_kernel, dim3(1), dim3(kSmallThreads), small_sm, s, topk_idx, (int)T, k, E,
-                           counts, offsets, perm_row, row_token, err);
+                           counts, offsets, perm_row, row_token, err, early_trigger ? 1 : 0);
         }
         if (e != cudaSuccess) return e;
         n = 1;
