@@ -241,6 +241,10 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
     const int nrows = offsets[E];
     const int lane = threadIdx.x & 31;
     const int vec = H / 8;
+    // each row of x is read k times and x fits in L2, while the T*k copies stream out once: keep
+    // x in L2 (evict-last) and let the copies pass through (evict-first), so the write stream
+    // does not push x out and make every copy re-read it from HBM
+    const uint64_t keep = l2_policy_evict_last(), pass = l2_policy_evict_first();
     for (int r = blockIdx.x * 8 + (threadIdx.x >> 5); r < nrows; r += gridDim.x * 8) {
         const int t = row_token[r];
         if (t < 0 || t >= T) {
@@ -253,11 +257,11 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
         for (; c + 224 < vec; c += 256) {   // eight 16-byte vectors in flight per lane
             uint4 v[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = __ldg(src + c + 32 * i);
+            for (int i = 0; i < 8; ++i) v[i] = ld_global_hint(src + c + 32 * i, keep);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) dst[c + 32 * i] = v[i];
+            for (int i = 0; i < 8; ++i) st_global_hint(dst + c + 32 * i, v[i], pass);
         }
-        for (; c < vec; c += 32) dst[c] = src[c];
+        for (; c < vec; c += 32) st_global_hint(dst + c, ld_global_hint(src + c, keep), pass);
     }
 }
 

@@ -253,15 +253,16 @@ router_topk_kernel(const float* __restrict__ part, int splits, const float* __re
         const uint32_t ml = __reduce_max_sync(0xFFFFFFFFu, bh == mh ? bl : 0u);
         const uint32_t ee = __reduce_min_sync(0xFFFFFFFFu, (bh == mh && bl == ml) ? (uint32_t)(lane + 32 * bi)
                                                                                    : 0xFFFFFFFFu);
+        // the winning lane clears the winner's key; written as selects over every slot so the
+        // arrays stay in registers (a store at a computed index would move them to local memory)
+        const int wq = ((int)(ee & 31u) == lane) ? (int)(ee >> 5) : -1;
         float sw = 0.f;
-        if ((int)(ee & 31u) == lane) {
 #pragma unroll
-            for (int q = 0; q < NPL; ++q)
-                if (q == (int)(ee >> 5)) {
-                    kh[q] = 0u;
-                    kl[q] = 0u;
-                    sw = S[q];
-                }
+        for (int q = 0; q < NPL; ++q) {
+            const bool hit = q == wq;
+            sw = hit ? S[q] : sw;
+            kh[q] = hit ? 0u : kh[q];
+            kl[q] = hit ? 0u : kl[q];
         }
         sw = __shfl_sync(0xFFFFFFFFu, sw, ee & 31u);
         if (lane == j) {
