@@ -269,6 +269,13 @@ SMOE_API smoe_status_t smoe_clear_device_error(void* ws, void* stream);
  * a misaligned pointer. (A library operation of its own; the pages have no counterpart.) */
 SMOE_API smoe_status_t smoe_selftest_wait_timeout(uint64_t limit_ns, uint64_t* elapsed_ns_opt, void* ws, void* stream);
 
+/* Self-test of the expert epilogue's arithmetic: out[i] = SiLU(g[i]) * u[i] for n elements,
+ * computed as the gate/up GEMM's epilogue computes it from its fp32 accumulators (fast exponential
+ * and reciprocal on the special-function unit). SiLU(z) = z / (1 + e^-z) is the expert
+ * activation (Step 3.5 Flash summary, paperlayer.ai, §B: SwiGLU gate and up projections). All
+ * pointers are device fp32 arrays of n elements, 16-byte aligned; asynchronous on the stream. */
+SMOE_API smoe_status_t smoe_selftest_swiglu(const float* g, const float* u, int64_t n, float* out, void* stream);
+
 /* Number of kernel launches the last successful call on this host thread enqueued. */
 SMOE_API int32_t smoe_last_launch_count(void);
 

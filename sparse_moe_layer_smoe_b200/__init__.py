@@ -85,6 +85,7 @@ _SIGS = {
     "smoe_workspace_bytes_fp8": ([_cfgp, _i64, ctypes.POINTER(_sz)], ctypes.c_int),
     "smoe_forward_fp8": ([_cfgp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "smoe_selftest_wait_timeout": ([ctypes.c_uint64, _vp, _vp, _vp], ctypes.c_int),
+    "smoe_selftest_swiglu": ([_vp, _vp, _i64, _vp, _vp], ctypes.c_int),
 }
 
 _lib = None
@@ -226,6 +227,11 @@ def smoe_forward_fp8(cfg, x, T, w_router, bias, packed_fp8, out, ws=None, ws_byt
     _check("smoe_forward_fp8", lib().smoe_forward_fp8(ctypes.byref(cfg), _p(x), T, _p(w_router), _p(bias),
                                                       _p(packed_fp8), _p(out), _p(ws), _ws_bytes(ws, ws_bytes),
                                                       _s(stream)))
+
+
+def smoe_selftest_swiglu(g, u, n, out, stream=None) -> None:
+    """The expert epilogue's SiLU(g) * u (see include/stepmoe.h)."""
+    _check("smoe_selftest_swiglu", lib().smoe_selftest_swiglu(_p(g), _p(u), int(n), _p(out), _s(stream)))
 
 
 def smoe_selftest_wait_timeout(limit_ns, elapsed_ns=None, ws=None, stream=None) -> None:

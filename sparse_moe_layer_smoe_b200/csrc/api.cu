@@ -433,6 +433,16 @@ smoe_status_t smoe_selftest_wait_timeout(uint64_t limit_ns, uint64_t* elapsed_ns
                                             static_cast<cudaStream_t>(stream)));
 }
 
+smoe_status_t smoe_selftest_swiglu(const float* g, const float* u, int64_t n, float* out, void* stream) {
+    if (n < 0) return SMOE_ERR_INVALID_ARG;
+    launches_reset();
+    if (n == 0) return SMOE_OK;
+    SMOE_REQUIRE_PTR(g);
+    SMOE_REQUIRE_PTR(u);
+    SMOE_REQUIRE_PTR(out);
+    return cuda_status(launch_swiglu_selftest(g, u, n, out, static_cast<cudaStream_t>(stream)));
+}
+
 smoe_status_t smoe_get_device_error(const void* ws, int32_t* code, void* stream) {
     if (ws == nullptr || code == nullptr) return SMOE_ERR_INVALID_ARG;
     int32_t v = 0;

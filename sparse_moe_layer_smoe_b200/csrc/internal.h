@@ -167,6 +167,9 @@ cudaError_t launch_pack(const smoe_config_t& c, const uint16_t* wg, const uint16
 // The bounded-wait self-test (smoe_selftest_wait_timeout).
 cudaError_t launch_wait_selftest(int32_t* err, uint64_t limit_ns, uint64_t* elapsed_ns, cudaStream_t s);
 
+// The expert epilogue's SiLU(g) * u (smoe_selftest_swiglu).
+cudaError_t launch_swiglu_selftest(const float* g, const float* u, int64_t n, float* out, cudaStream_t s);
+
 size_t packed_gateup_bytes(const smoe_config_t& c);
 size_t packed_down_bytes(const smoe_config_t& c);
 

@@ -24,7 +24,22 @@ __global__ void wait_timeout_selftest_kernel(int32_t* err, uint64_t limit_ns, ui
     if (ok) record_error(err, SMOE_ERR_DEVICE);   // cannot happen: nothing arrived
 }
 
+// The gate/up epilogue's SiLU(g) * u (silu_mul, as the GEMM epilogue computes it), one element
+// per thread.
+__global__ void swiglu_selftest_kernel(const float* g, const float* u, int64_t n, float* out) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) out[i] = silu_mul(g[i], u[i]);
+}
+
 }  // namespace
+
+cudaError_t launch_swiglu_selftest(const float* g, const float* u, int64_t n, float* out, cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    swiglu_selftest_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(g, u, n, out);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) launches_add(1);
+    return e;
+}
 
 cudaError_t launch_wait_selftest(int32_t* err, uint64_t limit_ns, uint64_t* elapsed_ns, cudaStream_t s) {
     wait_timeout_selftest_kernel<<<1, 32, 0, s>>>(err, limit_ns, elapsed_ns);
