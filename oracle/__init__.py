@@ -15,12 +15,12 @@ from .cpp import (bf16_to_f64, combine, f32_to_f64, moe_dense_masked, moe_given_
                   permute, route, router_logits, select_topk, sigmoid, silu, swiglu_ffn, swiglu_hidden,
                   valid_selections)
 from .diag import SUMMARY_FIELDS, Diagnostics, diagnostics, expert_output_norms, summarise
-from .fp8 import (E4M3_MAX, e4m3_code, e4m3_decode, e4m3_round, moe_sparse_fp8, quantize_rows, round_bf16,
-                  swiglu_ffn_fp8)
+from .fp8 import (E4M3_MAX, QuantExpert, e4m3_code, e4m3_decode, e4m3_round, moe_sparse_fp8, quantize_expert,
+                  quantize_rows, round_bf16, swiglu_ffn_fp8)
 from .moe import NEAR_TIE_EPS, Route
 
 __all__ = ["cpp", "moe", "SUMMARY_FIELDS", "Diagnostics", "diagnostics", "expert_output_norms", "summarise",
-           "E4M3_MAX", "e4m3_code", "e4m3_decode", "e4m3_round", "moe_sparse_fp8", "quantize_rows", "round_bf16",
+           "E4M3_MAX", "QuantExpert", "quantize_expert", "e4m3_code", "e4m3_decode", "e4m3_round", "moe_sparse_fp8", "quantize_rows", "round_bf16",
            "swiglu_ffn_fp8", "NEAR_TIE_EPS", "Route", "bf16_to_f64", "combine", "f32_to_f64", "moe_dense_masked",
            "moe_given_selection", "moe_sparse", "normalise", "permute", "route", "router_logits", "select_topk",
            "sigmoid", "silu", "swiglu_ffn", "swiglu_hidden", "valid_selections"]

@@ -31,7 +31,12 @@ E4M3_MAX = 448.0
 
 
 def e4m3_round(a: np.ndarray) -> np.ndarray:
-    """Nearest e4m3 value (ties to even mantissa), saturating at +-448; exact in fp64."""
+    """Nearest e4m3 value (ties to even mantissa), saturating at +-448; exact in fp64.
+
+    fp32 input takes an equivalent path on the bit pattern (the quantiser's inputs are fp32);
+    anything else the arithmetic one below."""
+    if isinstance(a, np.ndarray) and a.dtype == np.float32:
+        return _e4m3_round_f32(a)
     a = np.asarray(a, dtype=np.float64)
     mag = np.abs(a)
     # binade exponent, clamped at the subnormal range (the quantum there is 2^-9)
@@ -42,6 +47,23 @@ def e4m3_round(a: np.ndarray) -> np.ndarray:
     r = np.rint(mag / q) * q          # mag / q is exact (q a power of two); rint: half to even
     r = np.minimum(r, E4M3_MAX)
     return np.copysign(r, a)
+
+
+def _e4m3_round_f32(a: np.ndarray) -> np.ndarray:
+    """e4m3_round for fp32 values. In the normal e4m3 binades (|a| >= 2^-6) keeping 3 of fp32's
+    23 mantissa bits with round-to-nearest-even is integer arithmetic on the bit pattern: add
+    0x7FFFF plus the lowest kept bit, then clear the 20 dropped bits (a carry moves into the
+    exponent, as rounding up to the next binade should). Below 2^-6 the e4m3 quantum is 2^-9:
+    |a| * 2^9 is exact and rint rounds half to even. Then saturation at 448."""
+    u = a.view(np.uint32)
+    mag_u = u & np.uint32(0x7FFFFFFF)
+    lsb = (mag_u >> np.uint32(20)) & np.uint32(1)
+    rounded = ((mag_u + np.uint32(0x7FFFF) + lsb) & np.uint32(0xFFF00000)).view(np.float32).astype(np.float64)
+    mag = np.abs(a.astype(np.float64))
+    sub = mag < 2.0 ** -6
+    r = np.where(sub, np.rint(mag * 2.0 ** 9) * 2.0 ** -9, rounded)
+    r = np.minimum(r, E4M3_MAX)
+    return np.copysign(r, a.astype(np.float64))
 
 
 def e4m3_code(v: np.ndarray) -> np.ndarray:
@@ -77,7 +99,7 @@ def quantize_rows(a: np.ndarray):
     amax = np.max(np.abs(a32), axis=-1)
     s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
     scaled = (a32 / s[..., None]).astype(np.float32)
-    return e4m3_round(scaled), s
+    return e4m3_round(scaled), s   # fp32 in: the bit-pattern path
 
 
 def round_bf16(a: np.ndarray) -> np.ndarray:
@@ -88,12 +110,24 @@ def round_bf16(a: np.ndarray) -> np.ndarray:
     return r.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
-def swiglu_ffn_fp8(X: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray, limit: float = 0.0) -> np.ndarray:
-    """F_q(X) for rows X [n, H] with fp64 weights (bf16 values): reading 3."""
-    qx, sx = quantize_rows(X)
+class QuantExpert(tuple):
+    """An expert's weights already quantised per row (reading 2): (qg, sg, qu, su, qd, sd), the
+    values on the e4m3 grid as fp64 and the fp32 row scales. An ExpertFn may return one of these
+    instead of the bf16 weights, so that a caller can quantise each expert once."""
+
+
+def quantize_expert(Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray) -> QuantExpert:
     qg, sg = quantize_rows(Wg)
     qu, su = quantize_rows(Wu)
     qd, sd = quantize_rows(Wd)
+    return QuantExpert((qg, sg, qu, su, qd, sd))
+
+
+def swiglu_ffn_fp8(X: np.ndarray, Wg, Wu=None, Wd=None, limit: float = 0.0) -> np.ndarray:
+    """F_q(X) for rows X [n, H] with fp64 weights (bf16 values), or with one QuantExpert in place
+    of the three weights: reading 3."""
+    qg, sg, qu, su, qd, sd = Wg if isinstance(Wg, QuantExpert) else quantize_expert(Wg, Wu, Wd)
+    qx, sx = quantize_rows(X)
     sx64 = sx.astype(np.float64)[:, None]
     G = (qx @ qg.T) * sx64 * sg.astype(np.float64)[None, :]
     U = (qx @ qu.T) * sx64 * su.astype(np.float64)[None, :]
@@ -108,8 +142,11 @@ def swiglu_ffn_fp8(X: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray
 def moe_sparse_fp8(x: np.ndarray, r: Route, expert: ExpertFn, E: int, limit: float = 0.0,
                    limit_shared: float = 0.0) -> np.ndarray:
     """out[t] = F_q,shared(x_t) + sum_j w[t, j] F_q,idx[t, j](x_t) over the selected experts."""
-    out = swiglu_ffn_fp8(x, *expert(E), limit=limit_shared)
+    def weights(e):
+        w = expert(e)
+        return (w,) if isinstance(w, QuantExpert) else tuple(w)
+    out = swiglu_ffn_fp8(x, *weights(E), limit=limit_shared)
     for e in np.unique(r.idx):
         rows, slots = np.nonzero(r.idx == e)
-        out[rows] += r.w[rows, slots][:, None] * swiglu_ffn_fp8(x[rows], *expert(int(e)), limit=limit)
+        out[rows] += r.w[rows, slots][:, None] * swiglu_ffn_fp8(x[rows], *weights(int(e)), limit=limit)
     return out
