@@ -160,3 +160,19 @@ def test_pins_catch_scale_without_the_format_maximum(monkeypatch):
     with pytest.raises(AssertionError):
         test_quantize_rows_closed_forms()
     assert real is not bad
+
+
+def test_fp32_rounding_path_equals_the_arithmetic_one():
+    """e4m3_round of an fp32 array rounds on the bit pattern; it must give what the arithmetic
+    path gives for the same values in fp64: across the binades, the subnormals, saturation and
+    every midpoint between neighbouring e4m3 values (ties to even)."""
+    rng = np.random.default_rng(17)
+    a = (rng.standard_normal(200_000) * np.exp2(rng.integers(-14, 10, 200_000))).astype(np.float32)
+    grid = np.unique(np.abs(oracle.e4m3_decode(np.arange(256, dtype=np.uint8))))
+    grid = grid[np.isfinite(grid)]
+    mids = ((grid[:-1] + grid[1:]) / 2).astype(np.float32)
+    special = np.array([0.0, -0.0, 448, 449, 464, 480, 1e6, -1e6, 2.0 ** -10, -(2.0 ** -10)], dtype=np.float32)
+    for v in (a, mids, -mids, special):
+        fast = oracle.e4m3_round(v)
+        slow = oracle.e4m3_round(v.astype(np.float64))
+        assert np.array_equal(fast, slow) and np.array_equal(np.signbit(fast), np.signbit(slow))
