@@ -413,3 +413,38 @@ def test_forward_routing_collapse(T):
     fro, mx = assert_close(bf16_tensor_to_f64(out)[rows], ref, f"collapse T={T} forward (sampled tokens)")
     assert torch.isfinite(out.float()).all()
     print(f"collapse T={T}: rows={len(rows)} rel_fro={fro:.2e} rel_max={mx:.2e}")
+
+
+@pytest.mark.parametrize("T", [700, 1024, 1500])
+def test_forward_parity_mid_batches(T):
+    """Batch sizes between the named workloads, each on another launch plan: T = 700 (tensor-core
+    router, 32-token tiles with rows gathered inside the single-CTA GEMM), 1024 (CTA pairs with
+    64-token tiles, the one-CTA permutation at its limit) and 1500 (CTA pairs with 64-token tiles,
+    the multi-block permutation). The first T tokens of the prefill batch at the Step shape; the
+    whole layer against the oracle on 128 tokens spread over the batch."""
+    w0 = synth.WORKLOADS["prefill"]
+    w = synth.Workload("mid", T, w0.H, w0.E, w0.k, w0.I, w0.Is)
+    cfg = cfg_of(w)
+    _, _, wr, _, packed = device_inputs("prefill")
+    xh = synth.host_x_rows(w0, np.arange(T))
+    x = torch.from_numpy(xh.view(np.int16)).cuda().view(torch.bfloat16)
+    bias = torch.zeros(w.E, dtype=torch.float32, device="cuda")
+    out = torch.empty(T, w.H, dtype=torch.bfloat16, device="cuda")
+    ws = _ws(cfg, T, forward=True)
+    smoe.smoe_forward(cfg, x, T, wr, bias, packed, out, ws)
+    assert smoe.smoe_get_device_error(ws) == 0
+    idx = torch.empty(T, w.k, dtype=torch.int32, device="cuda")
+    wt = torch.empty(T, w.k, dtype=torch.float32, device="cuda")
+    smoe.smoe_route(cfg, x, T, wr, bias, idx, wt, None, _ws(cfg, T))
+    gi = idx.cpu().numpy()
+    x64 = oracle.bf16_to_f64(xh)
+    r = oracle.route(x64, oracle.f32_to_f64(synth.host_w_router(w0)), np.zeros(w.E), w.k, w.route_scale)
+    rows = sorted(t for t in stratified_tokens(T, 128, RNG) if not r.near_tie[t])
+    for t in rows:
+        ok, _ = selection_ok(r, t, tuple(sorted(gi[t].tolist())), w.k)
+        assert ok, f"token {t}"
+    sub = oracle.Route(r.logits[rows], r.s[rows], r.bhat[rows], r.idx[rows], r.w[rows], r.gap[rows])
+    ref = oracle.moe_sparse(x64[rows], sub, HostExperts(w0), w.E)
+    fro, mx = assert_close(bf16_tensor_to_f64(out)[rows], ref, f"T={T} forward (sampled tokens)")
+    assert torch.isfinite(out.float()).all()
+    print(f"T={T}: forward rows={len(rows)} rel_fro={fro:.2e} rel_max={mx:.2e}")
