@@ -394,5 +394,18 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
         : "memory");
 }
 
+// tile::gather4 for CTA pairs: four rows of a one-row-box map into this CTA's shared memory,
+// completing on the first CTA's barrier (as tma_load_2d_pair).
+__device__ __forceinline__ void tma_gather4_2d_pair(uint32_t dst, const CUtensorMap* map, int32_t c0, int32_t r0,
+                                                    int32_t r1, int32_t r2, int32_t r3, uint32_t bar_leader,
+                                                    uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar_leader),
+        "l"(policy)
+        : "memory");
+}
+
 }  // namespace smoe
 

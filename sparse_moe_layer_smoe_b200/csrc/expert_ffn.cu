@@ -56,6 +56,12 @@ constexpr int kMaxStages = SMOE_MAX_STAGES;
 #define SMOE_PAIR_MIN_TILE 64    // CTA pairs for launches whose largest token tile is at least this
 #endif
 constexpr int kPairMinTile = SMOE_PAIR_MIN_TILE;
+#ifndef SMOE_PAIR_EPI_WARPS
+#define SMOE_PAIR_EPI_WARPS 8    // epilogue warps of a CTA-pair gate/up CTA: 4, 8 or 16
+#endif
+#ifndef SMOE_PAIR_EPI_WARPS_DOWN
+#define SMOE_PAIR_EPI_WARPS_DOWN 8   // the same for the down GEMM
+#endif
 
 struct GemmMaps {
     CUtensorMap w;                  // weights [rows][K]: box {BK, 256 (gate/up) or 128 (down)}
@@ -98,6 +104,12 @@ struct GemmParams {
 
 // What a launch computes: the down projection, the fused gate/up + SiLU*mul, or router logits.
 enum GemmMode { MODE_DOWN = 0, MODE_GATEUP = 1, MODE_ROUTER = 2 };
+
+// CTA-pair kernels: producer warp, MMA warp and the epilogue warps of their mode
+template <int MODE>
+__host__ __device__ constexpr int pair_epi_warps() { return MODE == MODE_DOWN ? SMOE_PAIR_EPI_WARPS_DOWN : SMOE_PAIR_EPI_WARPS; }
+template <int MODE>
+__host__ __device__ constexpr int pair_threads() { return 64 + 32 * pair_epi_warps<MODE>(); }
 
 template <int MODE, int BK>
 struct GemmCfg {
@@ -255,15 +267,18 @@ __device__ int build_tile_table(const int32_t* offsets, int E, int T, int routed
 // Epilogue, part 1: drain this thread's accumulator row (one output feature, up to 256 token
 // columns) into registers as packed bf16 pairs: SiLU(gate) * up for gate/up (after the SwiGLU
 // clamp when lim > 0), the plain value for down. 32-column TMEM loads, one wait each.
-// nch = number of 32-column chunks holding valid tokens.
+// nch = number of 32-column chunks holding valid tokens. A thread takes the whole row (NS = 8) or,
+// where two epilogue warps share a quarter of the TMEM lanes, every other chunk: its chunk i is
+// accumulator chunk c0 + (8 / NS) i, and hv and cs are indexed by i.
 // With F8 (e4m3 operands) the accumulators are first scaled: by rs_g * s(col) (gate, or the down
 // output) and rs_u * s(col) (up), rs = this feature's weight-row scale and s(col) the activation
 // scale of the column, which lane j of the warp holds in cs[c] for column 32 c + j.
-template <bool DUAL, bool F8>
-__device__ __forceinline__ void epi_load(uint32_t t_row, int nt_max, int nch, float lim, uint32_t (&hv)[128],
-                                         float rs_g, float rs_u, const float (&cs)[8]) {
+template <bool DUAL, bool F8, int NS = 8>
+__device__ __forceinline__ void epi_load(uint32_t t_row, int nt_max, int nch, float lim, uint32_t (&hv)[16 * NS],
+                                         float rs_g, float rs_u, const float (&cs)[NS], int c0 = 0) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int i = 0; i < NS; ++i) {
+        const int c = c0 + (8 / NS) * i;
         if (c < nch) {
             uint32_t a[32], b[32];
             if (DUAL)
@@ -273,18 +288,18 @@ __device__ __forceinline__ void epi_load(uint32_t t_row, int nt_max, int nch, fl
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 float v0 = __uint_as_float(a[2 * j]), v1 = __uint_as_float(a[2 * j + 1]);
-                float c0 = 1.f, c1 = 1.f;
+                float s0 = 1.f, s1 = 1.f;
                 if (F8) {
-                    c0 = __shfl_sync(0xFFFFFFFFu, cs[c], 2 * j);
-                    c1 = __shfl_sync(0xFFFFFFFFu, cs[c], 2 * j + 1);
-                    v0 *= rs_g * c0;
-                    v1 *= rs_g * c1;
+                    s0 = __shfl_sync(0xFFFFFFFFu, cs[i], 2 * j);
+                    s1 = __shfl_sync(0xFFFFFFFFu, cs[i], 2 * j + 1);
+                    v0 *= rs_g * s0;
+                    v1 *= rs_g * s1;
                 }
                 if (DUAL) {
                     float u0 = __uint_as_float(b[2 * j]), u1 = __uint_as_float(b[2 * j + 1]);
                     if (F8) {
-                        u0 *= rs_u * c0;
-                        u1 *= rs_u * c1;
+                        u0 *= rs_u * s0;
+                        u1 *= rs_u * s1;
                     }
                     if (lim > 0.0f) {   // SwiGLU clamp: gate from above, up on both sides
                         v0 = fminf(v0, lim);
@@ -295,36 +310,40 @@ __device__ __forceinline__ void epi_load(uint32_t t_row, int nt_max, int nch, fl
                     v0 = silu_mul(v0, u0);
                     v1 = silu_mul(v1, u1);
                 }
-                hv[16 * c + j] = (uint32_t)float_to_bf16_bits(v0) | ((uint32_t)float_to_bf16_bits(v1) << 16);
+                hv[16 * i + j] = (uint32_t)float_to_bf16_bits(v0) | ((uint32_t)float_to_bf16_bits(v1) << 16);
             }
         }
     }
 }
 
 // Epilogue, part 2: store the valid token columns of this thread's feature (after the accumulator
-// has been handed back to the MMA thread).
-__device__ __forceinline__ void epi_store(const uint32_t (&hv)[128], int nch, int nvalid, uint16_t* out, size_t dst0,
-                                          int ld) {
+// has been handed back to the MMA thread); chunks as in epi_load.
+template <int NS = 8>
+__device__ __forceinline__ void epi_store(const uint32_t (&hv)[16 * NS], int nch, int nvalid, uint16_t* out,
+                                          size_t dst0, int ld, int c0 = 0) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int i = 0; i < NS; ++i) {
+        const int c = c0 + (8 / NS) * i;
         if (c < nch) {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
                 if (32 * c + j < nvalid)
-                    out[dst0 + (size_t)(32 * c + j) * ld] = (uint16_t)((j & 1) ? (hv[16 * c + j / 2] >> 16)
-                                                                               : (hv[16 * c + j / 2] & 0xFFFFu));
+                    out[dst0 + (size_t)(32 * c + j) * ld] = (uint16_t)((j & 1) ? (hv[16 * i + j / 2] >> 16)
+                                                                               : (hv[16 * i + j / 2] & 0xFFFFu));
         }
     }
 }
 
 // e4m3 launches: lane j loads the activation scale of columns 32 c + j of a unit (0 past its
-// valid rows); issued before the accumulator wait, so the loads overlap the MMAs.
+// valid rows) for the thread's chunks c (as in epi_load); issued before the accumulator wait, so
+// the loads overlap the MMAs.
+template <int NS = 8>
 __device__ __forceinline__ void load_col_scales(const GemmParams& p, const Unit& w, int nvalid, const int32_t* offs,
-                                                int lane, float (&cs)[8]) {
+                                                int lane, float (&cs)[NS], int c0 = 0) {
     const int base = (w.g < p.E ? offs[w.g] : p.scale_shared_base) + w.nb * w.nt;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const int col = 32 * c + lane;
+    for (int i = 0; i < NS; ++i) {
+        const int col = 32 * (c0 + (8 / NS) * i) + lane;
         float v = 0.f;
         if (col < nvalid) {
             int idx = base + col;
@@ -337,7 +356,7 @@ __device__ __forceinline__ void load_col_scales(const GemmParams& p, const Unit&
             }
             if (idx >= 0) v = p.act_scale[idx];
         }
-        cs[c] = v;
+        cs[i] = v;
     }
 }
 
@@ -675,6 +694,13 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
 // loads in full. Work unit = (token tile, 256-feature block), dealt to the pairs in the same
 // snake order as the single-CTA kernel's units.
 //
+// Roles (320 threads per CTA): warp 0 loads (lane 0; all lanes issue the row gathers in gather
+// mode), warp 1 lane 0 of the first CTA issues the MMAs, and warps 2-9 drain the accumulator,
+// two warps per quarter of the TMEM lanes, each taking every other 32-column chunk. Two drain
+// warps per SM sub-partition cut the prefill step's down GEMM by ~10% against one (the single
+// drain warp's TMEM-load waits and 2-byte column stores did not hide behind the next unit's
+// MMAs); four per quarter measured no faster.
+//
 // Signals: both CTAs' loads complete on the first CTA's stage barrier (it arms the expected
 // bytes of both); the first CTA's MMA thread commits stage-free and accumulator-ready to each
 // CTA's barrier; both CTAs' epilogue warps arrive on the first CTA's accumulator-free barrier.
@@ -682,7 +708,7 @@ expert_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
 // pair's MMAs are done.
 // ------------------------------------------------------------------------------------------
 template <int MODE, int BK, bool F8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<MODE>(), 1)
 expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     using C = GemmCfg<MODE, BK>;
     constexpr bool DUAL = C::DUAL;
@@ -720,7 +746,7 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&tfull[a]), 1);
-            mbar_init(smem_u32(&tempty[a]), 8);   // 4 epilogue warps x 2 CTAs
+            mbar_init(smem_u32(&tempty[a]), 2 * pair_epi_warps<MODE>());   // epilogue warps of both CTAs
         }
         mbar_init(smem_u32(drain), 1);
         *abort_flag = 0;
@@ -754,8 +780,15 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
     const uint32_t tmem_base = *tmem_slot;
     const int total = *ntiles_slot * MBP;   // units: (token tile, 256-feature block)
 
-    if (warp == 0 && lane == 0) {
+    // gather mode (row_token set): all 32 lanes of warp 0 issue row gathers; otherwise lane 0 alone
+    const unsigned pmask = (p.row_token != nullptr) ? 0xFFFFFFFFu : 1u;
+    if (warp == 0 && ((pmask >> lane) & 1u)) {
         // ---------------------------------------------------------------- TMA producer (both CTAs)
+        // Lane 0 waits for a free stage, arms the barrier (first CTA) and loads this CTA's weight
+        // tile. Its half of the token rows comes as one tile (contiguous rows), or, for routed
+        // groups in gather mode, as rows picked out of x by tile::gather4 loads, lane c taking
+        // rows 4c..4c+3 of the half (rows past the group's end repeat its last row; the MMA never
+        // reads them).
         const uint64_t pol_w = l2_policy_evict_first();
         const uint64_t pol_a = l2_policy_evict_last();
         int stage = 0;
@@ -773,30 +806,47 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
             const int n_mma = mma_cols(group_rows(w.g, E, p.T, offs) - w.nb * w.nt, w.nt);
             const int b_row = (w.g < E ? offs[w.g] : p.shared_in_row) + w.nb * w.nt + (int)rank * (n_mma / 2);
             const int ti = tile_index(w.nt);
-            const CUtensorMap* bm = (w.g < E) ? &maps.act[ti] : &maps.sh[ti];
+            const bool gather = p.row_token != nullptr && w.g < E;
+            const CUtensorMap* bm = (w.g < E) ? &maps.act[gather ? 0 : ti] : &maps.sh[ti];
             const uint32_t tx = (uint32_t)(2 * (C::A_BYTES + half * BK * 2));
             const uint64_t pw = weight_policy(group_rows(w.g, E, p.T, offs), w.nt, pol_w, pol_a);
+            const bool my_chunk = gather && lane < half / 4;
+            int tok[4] = {0, 0, 0, 0};
+            if (my_chunk) {
+                const int last = offs[w.g + 1] - 1;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) tok[r] = p.row_token[min(b_row + 4 * lane + r, last)];
+            }
             for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag, true)) { ok = false; break; }
+                if (lane == 0) ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag, true);
+                ok = __shfl_sync(pmask, ok, 0);
+                if (!ok) break;
                 const uint32_t fb_local = smem_u32(&full[stage]);
                 const uint32_t fb_leader = mapa_shared(fb_local, 0);
-                if (rank == 0) mbar_arrive_expect_tx(fb_local, tx);
                 uint8_t* a_s = tiles + (size_t)stage * STAGE_B;
-                int wx, wy;
-                weight_tile_xy<EK, TK>(a_blk, kb, p.K, C::A_ROWS, wx, wy);
-                tma_load_2d_pair(smem_u32(a_s), &maps.w, wx, wy, fb_leader, pw);
-                tma_load_2d_pair(smem_u32(a_s + C::A_BYTES), bm, kb * EK, b_row, fb_leader, pol_a);
+                if (lane == 0) {
+                    if (rank == 0) mbar_arrive_expect_tx(fb_local, tx);
+                    int wx, wy;
+                    weight_tile_xy<EK, TK>(a_blk, kb, p.K, C::A_ROWS, wx, wy);
+                    tma_load_2d_pair(smem_u32(a_s), &maps.w, wx, wy, fb_leader, pw);
+                    if (!gather) tma_load_2d_pair(smem_u32(a_s + C::A_BYTES), bm, kb * EK, b_row, fb_leader, pol_a);
+                }
+                __syncwarp(pmask);
+                if (my_chunk)
+                    tma_gather4_2d_pair(smem_u32(a_s + C::A_BYTES + lane * 4 * BK * 2), bm, kb * EK, tok[0], tok[1],
+                                        tok[2], tok[3], fb_leader, pol_a);
                 armed |= 1u << stage;
                 armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                 if (++stage == S) { stage = 0; phase ^= 1u; }
             }
         }
-        if (rank == 0) {
+        if (rank == 0 && lane == 0) {
             // both CTAs' bytes of every armed stage are counted here: wait for them to land
             for (int s = 0; s < S; ++s)
                 if ((armed >> s) & 1u)
                     mbar_wait(smem_u32(&full[s]), (armed_par >> s) & 1u, p.err, abort_flag, false);
         }
+        __syncwarp(pmask);
     } else if (warp == 1 && lane == 0 && rank == 0) {
         // ---------------------------------------------------------------- MMA issuer (first CTA)
         const uint32_t idesc0 = F8 ? idesc_e4m3_f32(256, 0) : idesc_bf16_f32(256, 0);
@@ -854,7 +904,13 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
         mbar_wait(smem_u32(drain), 0u, p.err, abort_flag, false);
     } else if (warp >= 2) {
         // ---------------------------------------------------------------- epilogue (both CTAs)
+        // warp w reads TMEM lanes 32 (w % 4)..+31; with G = 1, 2 or 4 epilogue warps per lane
+        // quarter, warp group c0 = (w - 2) / 4 takes the 32-column chunks c0, c0 + G, ...
+        constexpr int G = pair_epi_warps<MODE>() / 4;
+        static_assert(G == 1 || G == 2 || G == 4, "1, 2 or 4 epilogue warps per TMEM lane quarter");
+        constexpr int NS = 8 / G;
         const int q = warp & 3;
+        const int c0 = (warp - 2) >> 2;
         const int row = q * 32 + lane;
         int acc = 0;
         uint32_t acc_phase = 0;
@@ -865,25 +921,26 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
             const int rows = group_rows(w.g, E, p.T, offs);
             const int out_base = (w.g < E ? offs[w.g] : p.shared_out_row) + w.nb * w.nt;
             const int nvalid = min(w.nt, rows - w.nb * w.nt);
-            float cs[8];
-            if (F8) load_col_scales(p, w, nvalid, offs, lane, cs);
+            float cs[NS];
+            if (F8) load_col_scales<NS>(p, w, nvalid, offs, lane, cs, c0);
             if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.err, abort_flag, true)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
             const int f = w.mb * 256 + (int)rank * 128 + row;
             const size_t dst0 = (size_t)out_base * p.out_ld + f;
             const int nch = (nvalid + 31) / 32;
-            uint32_t hv[128];
+            uint32_t hv[16 * NS];
             float rs_g = 1.f, rs_u = 1.f;
             if (F8) {
                 rs_g = p.w_scale[(size_t)(DUAL ? 2 * w.g : w.g) * p.n_out + f];
                 if (DUAL) rs_u = p.w_scale[(size_t)(2 * w.g + 1) * p.n_out + f];
             }
-            epi_load<DUAL, F8>(t_row, p.nt_max, nch, w.g < E ? p.clamp_routed : p.clamp_shared, hv, rs_g, rs_u, cs);
+            epi_load<DUAL, F8, NS>(t_row, p.nt_max, nch, w.g < E ? p.clamp_routed : p.clamp_shared, hv, rs_g, rs_u, cs,
+                                   c0);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));   // accumulator free
-            epi_store(hv, nch, nvalid, p.out, dst0, p.out_ld);
+            epi_store<NS>(hv, nch, nvalid, p.out, dst0, p.out_ld, c0);
             if (NACC == 2) {
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
@@ -1042,7 +1099,7 @@ cudaError_t run_gemm_pair(const GemmMaps& maps, GemmParams p, int num_sms, cudaS
     if (max_clusters[MODE] == 0) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(num_sms & ~1);
-        cfg.blockDim = dim3(kThreads);
+        cfg.blockDim = dim3(pair_threads<MODE>());
         cfg.dynamicSmemBytes = smem;
         int n = 0;
         e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
@@ -1052,7 +1109,7 @@ cudaError_t run_gemm_pair(const GemmMaps& maps, GemmParams p, int num_sms, cudaS
     const int pairs = std::min(num_sms / 2, max_clusters[MODE]);
     {
         LaunchTimer lt(MODE == MODE_GATEUP ? K_EXPERT_GATEUP : K_EXPERT_DOWN, s);
-        return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), smem, s, maps, p);
+        return launch_pdl(kern, dim3(2 * pairs), dim3(pair_threads<MODE>()), smem, s, maps, p);
     }
 }
 
@@ -1103,7 +1160,7 @@ cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const u
     GemmMaps m1, m2;
     const bool gather = x_perm == nullptr;
     // CTA pairs for large token tiles (each pair handles 256 output features)
-    const bool pairs = !gather && nt >= kPairMinTile && I % 256 == 0 && H % 256 == 0;
+    const bool pairs = nt >= kPairMinTile && I % 256 == 0 && H % 256 == 0;
     auto act_maps = [&](CUtensorMap* maps, const void* base, uint64_t rows, uint64_t cols) {
         return pairs ? make_half_act_maps(maps, base, rows, cols, nt, BK) : make_act_maps(maps, base, rows, cols, nt, BK);
     };
@@ -1120,7 +1177,7 @@ cudaError_t launch_expert_ffn(const smoe_config_t& c, const uint16_t* x, const u
 
     GemmParams p1{offsets, E, (int)T, (int)routed, H, I, 0, (int)routed, nt, 0, 0, I, I, gather ? row_token : nullptr,
                   c.swiglu_limit, c.swiglu_limit_shared, 1, 0, h, nullptr, err};
-    p1.shared_first = gather && SMOE_SHARED_FIRST ? 1 : 0;
+    p1.shared_first = gather && !pairs && SMOE_SHARED_FIRST ? 1 : 0;
     p1.shared_prewait = gather && !pairs && shared_prewait && shared_prewait_fits(c, T, num_sms) ? 1 : 0;
     cudaError_t e = pairs ? run_gemm_pair<MODE_GATEUP>(m1, p1, num_sms, s) : run_gemm<MODE_GATEUP>(m1, p1, num_sms, s);
     if (e != cudaSuccess) return e;
@@ -1144,7 +1201,7 @@ cudaError_t launch_expert_ffn_fp8(const smoe_config_t& c, const uint8_t* x_q, co
 
     GemmMaps m1, m2;
     const bool gather = x_q_perm == nullptr;
-    const bool pairs = !gather && nt >= kPairMinTile && I % 256 == 0 && H % 256 == 0;
+    const bool pairs = nt >= kPairMinTile && I % 256 == 0 && H % 256 == 0;
     auto act_maps = [&](CUtensorMap* maps, const void* base, uint64_t rows, uint64_t cols) {
         return pairs ? make_half_act_maps(maps, base, rows, cols, nt, BK, true)
                      : make_act_maps(maps, base, rows, cols, nt, BK, true);
@@ -1166,7 +1223,7 @@ cudaError_t launch_expert_ffn_fp8(const smoe_config_t& c, const uint8_t* x_q, co
     p1.act_scale = s_x;
     p1.scale_tok = row_token;
     p1.scale_shared_base = 0;
-    p1.shared_first = gather && SMOE_SHARED_FIRST ? 1 : 0;
+    p1.shared_first = gather && !pairs && SMOE_SHARED_FIRST ? 1 : 0;
     cudaError_t e = pairs ? run_gemm_pair<MODE_GATEUP, true>(m1, p1, num_sms, s)
                           : run_gemm<MODE_GATEUP, true>(m1, p1, num_sms, s);
     if (e != cudaSuccess) return e;
