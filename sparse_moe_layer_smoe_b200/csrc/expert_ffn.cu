@@ -939,7 +939,9 @@ expert_gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams 
                                    c0);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));   // accumulator free
+            // accumulator free: every lane's TMEM loads have completed (tcgen05.wait::ld), so the
+            // arrive needs no release; a release would first wait for the previous unit's stores
+            if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&tempty[acc]), 0));
             epi_store<NS>(hv, nch, nvalid, p.out, dst0, p.out_ld, c0);
             if (NACC == 2) {
                 acc ^= 1;

@@ -237,12 +237,17 @@ WORKLOADS = {
     # profiling case: the decode kernel shape (~2 rows per expert) on 32 experts, ~1 GB of weights
     "decode_e32": Workload("decode_e32", 8, 4096, 32, 8, 1280, 1280,
                            description="decode-shaped small case for counter captures: T=8, 32 experts top-8"),
-    # profiling case: the prefill kernel shape (~225 rows per expert, token tile 256) on 32 experts
     # experiment case: the prefill GEMM shape with operands mostly L2-resident (8 experts x 2048 rows)
     "gemm_l2": Workload("gemm_l2", 8192, 4096, 8, 2, 1280, 1280,
                         description="8 experts top-2 over 8192 tokens: ~2048 rows per expert, weights reused from L2"),
+    # profiling case: the prefill kernel shape (~225 rows per expert, token tile 256) on 32 experts
     "prefill_e32": Workload("prefill_e32", 900, 4096, 32, 8, 1280, 1280,
                             description="prefill-shaped small case for counter captures: T=900, 32 experts top-8"),
+    # profiling case: the prefill kernel shape (~228 rows per expert, one 256-row tile each) with
+    # several rounds of units per pair: 72 experts over 2048 tokens, ~2.6 GB on the device
+    "prefill_e72": Workload("prefill_e72", 2048, 4096, 72, 8, 1280, 1280,
+                            description="prefill-shaped steady-state case for counter captures: T=2048, 72 experts "
+                                        "top-8"),
     # profiling case: the skewed batch's kernel shape (mean ~114 rows per expert, Zipf popularity
     # with 16 dead experts, 1-row to multi-tile groups) on 72 experts, ~2.3 GB of weights
     "skewed_e72": Workload("skewed_e72", 1024, 4096, 72, 8, 1280, 1280, bias="zipf",
