@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(256, 3) combine_kernel(const uint16_t* __restr
         uint32_t* ou = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            ou[i] = (uint32_t)float_to_bf16_bits(acc[2 * i]) | ((uint32_t)float_to_bf16_bits(acc[2 * i + 1]) << 16);
+            ou[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
         reinterpret_cast<uint4*>(out)[(size_t)t * vec + c] = o;
     }
     if constexpr (NORMS) {

@@ -29,6 +29,14 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
+// Two fp32 values rounded to bf16 (nearest even) and packed, lo in the low half: one paired
+// conversion instead of two single ones and a pack (the single conversions share a slow pipe
+// with the SFU, which limited the down GEMM's drain).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return (uint32_t)__bfloat16_as_ushort(v.x) | ((uint32_t)__bfloat16_as_ushort(v.y) << 16);
+}
+
 // e4m3 code of an fp32 value: round to nearest even, finite values beyond +-448 saturate.
 __device__ __forceinline__ uint8_t float_to_e4m3(float f) {
     return (uint8_t)__nv_cvt_float_to_fp8(f, __NV_SATFINITE, __NV_E4M3);

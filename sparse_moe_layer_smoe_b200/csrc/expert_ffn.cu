@@ -310,7 +310,7 @@ __device__ __forceinline__ void epi_load(uint32_t t_row, int nt_max, int nch, fl
                     v0 = silu_mul(v0, u0);
                     v1 = silu_mul(v1, u1);
                 }
-                hv[16 * i + j] = (uint32_t)float_to_bf16_bits(v0) | ((uint32_t)float_to_bf16_bits(v1) << 16);
+                hv[16 * i + j] = pack_bf16x2(v0, v1);
             }
         }
     }
