@@ -30,8 +30,8 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
 }
 
 // Two fp32 values rounded to bf16 (nearest even) and packed, lo in the low half: one paired
-// conversion instead of two single ones and a pack (the single conversions share a slow pipe
-// with the SFU, which limited the down GEMM's drain).
+// conversion instead of two single ones and a pack (the single conversions issue on the XU
+// pipe, which the SFU's exp and reciprocal also use).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return (uint32_t)__bfloat16_as_ushort(v.x) | ((uint32_t)__bfloat16_as_ushort(v.y) << 16);
