@@ -146,7 +146,9 @@ SMOE_API smoe_status_t smoe_permute(const smoe_config_t* cfg, const int32_t* top
  * over their rows; group E is the shared expert over all T rows of x.
  *   x         [T][H] bf16
  *   x_perm    [T*k][H] bf16 rows grouped by offsets, or NULL: then the routed rows are read
- *             straight from x through row_token (TMA row gathers; no permuted copy of x)
+ *             straight from x through row_token (TMA row gathers; no permuted copy of x).
+ *             The results are the same either way; with token tiles above 32 rows the row
+ *             gathers are slower than loading x_perm (smoe_forward builds x_perm there).
  *   row_token [T*k] int32, as written by smoe_permute (needed when x_perm is NULL)
  *   offsets   [E+1] int32 (device), as written by smoe_permute
  *   packed    packed weights (smoe_pack_weights)
