@@ -44,6 +44,9 @@ namespace {
 #ifndef SMOE_MAX_TOKEN_TILE
 #define SMOE_MAX_TOKEN_TILE 256  // cap on the token tile (a tuning constant)
 #endif
+// 256 is also the largest MMA N, the largest box height of a TMA map (kNumTiles maps, 16..256),
+// and the most rows the producer warp's lanes cover with one four-row gather each per CTA half
+static_assert(SMOE_MAX_TOKEN_TILE >= 16 && SMOE_MAX_TOKEN_TILE <= 256, "token tile cap in 16..256");
 
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
