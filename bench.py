@@ -53,6 +53,9 @@ def parse_args(argv=None):
                    help="comma list of further workloads of the same layer shape timed in the same run and "
                         "reported under 'workloads' ('none': the headline only)")
     p.add_argument("--pct-steps", type=int, default=50, help="steps of the per-step spread pass (p10/p50/p90)")
+    p.add_argument("--cooldown", type=float, default=2.0,
+                   help="idle seconds before each workload after the headline, so that each one starts from the "
+                        "same power state instead of inheriting the previous workload's")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=4)
@@ -357,6 +360,10 @@ def measure(smoe, w, packed, args, dev, headline: bool):
                "min_count_live": int(live.min().item()) if touched else 0, "mean_count": T * w.k / E}
 
     # ---- device-resident timing (value)
+    if not headline and args.cooldown > 0:
+        # the 1 kW power cap lowers the clock after a tensor-heavy workload for a while: idle first
+        torch.cuda.synchronize()
+        time.sleep(args.cooldown)
     for _ in range(args.warmup):
         forward(x)
     torch.cuda.synchronize()
@@ -510,7 +517,7 @@ def run_ours(args):
             "config": entry["config"], "layer": entry["layer"], "experts": entry["experts"],
             "step_ms": entry["step_ms"], "kernels_ms_per_step": entry["kernels_ms_per_step"],
             "roofline": entry["roofline"], "e2e": entry["e2e"], "gpu_launches": entry["gpu_launches"],
-            "clocks": entry["clocks"],
+            "clocks": entry["clocks"], "cooldown_s": args.cooldown,
             "workloads": {n: {kk: vv for kk, vv in e.items() if kk != "config"} | {"T": synth.WORKLOADS[n].T}
                           for n, (e, _) in results.items()}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
