@@ -5,7 +5,8 @@
 * smoe_forward_fp8: the layer vs the oracle's e4m3 layer within the layer tolerances (relative
   Frobenius <= 1e-2, max |err| <= 2e-2 max|ref|): all tokens of the tiny layer, >= 256 tokens
   spread over the batch (spike rows included) at decode (gather mode), MTP, prefill and the Zipf-skewed batch (CTA
-  pairs, permuted e4m3 rows; skewed mixes 1-row and multi-tile groups);
+  pairs, permuted e4m3 rows; skewed mixes 1-row and multi-tile groups), and 128 tokens of a
+  1024-token batch (CTA pairs with 64-token tiles);
   the quantisation error against the bf16 oracle is printed for reference;
 * deterministic: two calls give the same bits.
 """
@@ -152,3 +153,32 @@ def test_forward_fp8_deterministic_and_ragged():
     w, x, *_ = device_inputs("decode")
     _, c = _forward_fp8("decode", x=x[:37].contiguous(), T=37)
     assert torch.isfinite(c.float()).all()
+
+
+def test_forward_fp8_mid_batch():
+    """T = 1024 (the first tokens of the prefill batch): the e4m3 GEMMs on CTA pairs with 64-token
+    tiles, every drain warp taking one or two 32-column chunks; 128 tokens spread over the batch
+    against the e4m3 oracle."""
+    T = 1024
+    w0 = synth.WORKLOADS["prefill"]
+    w = synth.Workload("mid_fp8", T, w0.H, w0.E, w0.k, w0.I, w0.Is)
+    cfg = cfg_of(w)
+    _, _, wr, _, _ = device_inputs("prefill")
+    xh = synth.host_x_rows(w0, np.arange(T))
+    x = torch.from_numpy(xh.view(np.int16)).cuda().view(torch.bfloat16)
+    bias = torch.zeros(w.E, dtype=torch.float32, device="cuda")
+    out = torch.empty(T, w.H, dtype=torch.bfloat16, device="cuda")
+    ws = smoe.workspace(cfg, T, fp8=True)
+    smoe.smoe_forward_fp8(cfg, x, T, wr, bias, _packed_fp8(w0), out, ws)
+    assert smoe.smoe_get_device_error(ws) == 0
+    x64 = oracle.bf16_to_f64(xh)
+    r = oracle.route(x64, oracle.f32_to_f64(synth.host_w_router(w0)), np.zeros(w.E), w.k, w.route_scale)
+    rows = sorted(t for t in stratified_tokens(T, 128, RNG) if not r.near_tie[t])
+    sub = oracle.Route(r.logits[rows], r.s[rows], r.bhat[rows], r.idx[rows], r.w[rows], r.gap[rows])
+    need = sorted(set(np.unique(sub.idx).tolist()) | {w.E})
+    with ThreadPoolExecutor(max_workers=8) as pool:
+        list(pool.map(lambda e: _quant_expert(w0, e), need))
+    ref8 = oracle.moe_sparse_fp8(x64[rows], sub, lambda e: _quant_expert(w0, e), w.E)
+    fro, mx = assert_close(bf16_tensor_to_f64(out)[rows], ref8, f"T={T} e4m3 forward vs e4m3 oracle")
+    assert torch.isfinite(out.float()).all()
+    print(f"T={T}: e4m3 forward rows={len(rows)} rel_fro={fro:.2e} rel_max={mx:.2e}")
