@@ -275,7 +275,7 @@ __device__ int build_tile_table(const int32_t* offsets, int E, int T, int routed
 // accumulator chunk c0 + (8 / NS) i, and hv and cs are indexed by i.
 // With F8 (e4m3 operands) the accumulators are first scaled: by rs_g * s(col) (gate, or the down
 // output) and rs_u * s(col) (up), rs = this feature's weight-row scale and s(col) the activation
-// scale of the column, which lane j of the warp holds in cs[c] for column 32 c + j.
+// scale of the column, which lane j of the warp holds in cs[i] for column 32 c + j of chunk i.
 template <bool DUAL, bool F8, int NS = 8>
 __device__ __forceinline__ void epi_load(uint32_t t_row, int nt_max, int nch, float lim, uint32_t (&hv)[16 * NS],
                                          float rs_g, float rs_u, const float (&cs)[NS], int c0 = 0) {
